@@ -1,0 +1,259 @@
+"""Plain CPU oracle for the 4-bit blocked weight matmul and the int8 tied LM head.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or link
+this module: only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` use it. It shares no code with the CUDA library; the two
+meet only through the seeded input generators, which hold none of the method's
+arithmetic.
+
+What it follows
+---------------
+* "ONNX export, quantization and the browser runtime" (tokenling docs),
+  section "Quantization (train/quantize.py)":
+    - step 1 (``gemm_to_matmul``): every body weight is a plain [K, N]
+      constant, K = in-features, N = out-features, so y = x @ W;
+    - step 2 (``dq4``): each body weight is stored 4-bit asymmetric, in blocks
+      of 32 along K, with an fp32 scale and a uint4 zero point per block (and
+      column), as raw packed UINT4 tensors, restored to fp32 by one blocked
+      DequantizeLinear:  w = (q - zp) * scale;
+    - step 3 (``embedding_int8``): the tied embedding / LM head is int8 with
+      one scale per token, in the head's [768, V] layout;
+    - step 4 (``last_token_logits``): the head runs on the last position only.
+  The same page's output list says "4-bit body, 8-bit embedding, fp32 compute".
+
+Readings where the page is silent (each is listed in the design notes):
+* nibble order: element i of a flat row-major tensor sits in byte i >> 1, in
+  the low nibble when i is even (the ONNX UINT4 packing, low nibble first);
+* zero points use the same packing over their [K/32, N] tensor;
+* scales are fp32 [K/32, N] row-major;
+* K must be a multiple of 32 and N even; anything else is rejected;
+* dequantisation is exact in (q - zp) and then one fp32 multiply rounded to
+  nearest-even, which is what DequantizeLinear computes in fp32;
+* the head has no zero point (symmetric) and no bias.
+
+Accumulation is fp64. Every function also returns sum_k |x_k * w_kn| so that
+callers can apply the tolerance |y - y_ref| <= 1e-5 * sum|x*w| + 1e-6.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK = 32  # K-block length of the 4-bit format (dq4: "blocks of 32 along K")
+ABS_TOL = 1e-6
+REL_TOL = 1e-5
+
+
+# --------------------------------------------------------------------------
+# nibble packing: "raw packed UINT4 tensors", two per byte, low nibble first
+# --------------------------------------------------------------------------
+
+def unpack_nibbles(packed, count: int) -> np.ndarray:
+    """Return the first ``count`` uint4 values (as uint8 0..15) of a packed buffer.
+
+    Element i is the low nibble of byte i >> 1 when i is even and the high
+    nibble when i is odd.
+    """
+    b = np.ascontiguousarray(packed, dtype=np.uint8).reshape(-1)
+    if count < 0 or count > 2 * b.size:
+        raise ValueError(f"cannot unpack {count} nibbles from {b.size} bytes")
+    out = np.empty(2 * b.size, dtype=np.uint8)
+    out[0::2] = b & 0x0F
+    out[1::2] = b >> 4
+    return out[:count]
+
+
+def pack_nibbles(q) -> np.ndarray:
+    """Pack uint4 values (0..15) two per byte, low nibble first.
+
+    An odd count leaves the high nibble of the last byte at zero.
+    """
+    v = np.ascontiguousarray(q).reshape(-1)
+    if v.size and (v.min() < 0 or v.max() > 15):
+        raise ValueError("uint4 values must lie in 0..15")
+    v = v.astype(np.uint8)
+    if v.size % 2:
+        v = np.concatenate([v, np.zeros(1, np.uint8)])
+    return (v[0::2] | (v[1::2] << 4)).astype(np.uint8)
+
+
+# --------------------------------------------------------------------------
+# 4-bit body weights
+# --------------------------------------------------------------------------
+
+def _rows(x, K: int) -> np.ndarray:
+    """x as fp64 [M, K] rows (a 1-D x of length K is one row)."""
+    a = np.asarray(x, dtype=np.float32)
+    if a.ndim == 1:
+        a = a.reshape(1, -1)
+    if a.ndim != 2 or a.shape[1] != K:
+        raise ValueError(f"x must be [M, {K}], got {a.shape}")
+    return a.astype(np.float64)
+
+
+def check_w4_shape(K: int, N: int) -> None:
+    if K < 0 or N < 0:
+        raise ValueError("negative shape")
+    if K % BLOCK:
+        raise ValueError(f"K={K} is not a multiple of {BLOCK}")
+    if N % 2:
+        raise ValueError(f"N={N} is odd")
+
+
+def dequantize_w4(qw, scales, zp, K: int, N: int) -> np.ndarray:
+    """Blocked DequantizeLinear of one [K, N] weight: fp32 w = (q - zp) * s.
+
+    ``qw`` holds K*N packed nibbles (flat [K, N] order), ``zp`` holds
+    (K/32)*N packed nibbles (flat [K/32, N] order) and ``scales`` is fp32
+    [K/32, N]. Row k uses block b = k // 32.
+    """
+    check_w4_shape(K, N)
+    nb = K // BLOCK
+    q = unpack_nibbles(qw, K * N).reshape(K, N).astype(np.int32)
+    z = unpack_nibbles(zp, nb * N).reshape(nb, N).astype(np.int32)
+    s = np.ascontiguousarray(scales, dtype=np.float32).reshape(nb, N)
+    blk = np.arange(K) // BLOCK
+    diff = (q - z[blk, :]).astype(np.float32)  # small integers: exact in fp32
+    return diff * s[blk, :]  # one fp32 multiply, round to nearest even
+
+
+def dequantize_w4_columns(qw, scales, zp, K: int, N: int, cols) -> np.ndarray:
+    """Columns ``cols`` of the dequantised [K, N] weight, without the rest.
+
+    Column n of row k is nibble k*N + n; with N even that is byte
+    k*(N/2) + n//2, low nibble when n is even.
+    """
+    check_w4_shape(K, N)
+    cols = np.asarray(cols, dtype=np.int64).reshape(-1)
+    nb = K // BLOCK
+    rows_q = np.ascontiguousarray(qw, dtype=np.uint8).reshape(K, N // 2)
+    rows_z = np.ascontiguousarray(zp, dtype=np.uint8).reshape(nb, N // 2)
+    s = np.ascontiguousarray(scales, dtype=np.float32).reshape(nb, N)
+    byte_q = rows_q[:, cols // 2]
+    byte_z = rows_z[:, cols // 2]
+    odd = (cols % 2).astype(bool)
+    q = np.where(odd[None, :], byte_q >> 4, byte_q & 0x0F).astype(np.int32)
+    z = np.where(odd[None, :], byte_z >> 4, byte_z & 0x0F).astype(np.int32)
+    blk = np.arange(K) // BLOCK
+    diff = (q - z[blk, :]).astype(np.float32)
+    return diff * s[blk][:, cols]
+
+
+def w4_matmul_ref(x, qw, scales, zp, K: int, N: int):
+    """y = x @ W for the whole output, fp64 accumulation.
+
+    Returns ``(y, a)`` with y = sum_k x_mk * w_kn and a = sum_k |x_mk * w_kn|,
+    both fp64 [M, N]. The inputs are read as fp32 and widened exactly.
+    """
+    w = dequantize_w4(qw, scales, zp, K, N).astype(np.float64)
+    x64 = _rows(x, K)
+    return x64 @ w, np.abs(x64) @ np.abs(w)
+
+
+def w4_matmul_ref_entries(x, qw, scales, zp, K: int, N: int, rows, cols):
+    """Sampled outputs y[rows[i], cols[i]] (and a[...]) for shapes too large to
+    dequantise whole. Only the named columns are dequantised."""
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1)
+    cols = np.asarray(cols, dtype=np.int64).reshape(-1)
+    ucols, inv = np.unique(cols, return_inverse=True)
+    w = dequantize_w4_columns(qw, scales, zp, K, N, ucols).astype(np.float64)
+    x64 = _rows(x, K)
+    xr = x64[rows]  # [S, K]
+    wc = w[:, inv].T  # [S, K]
+    return np.einsum("sk,sk->s", xr, wc), np.einsum("sk,sk->s", np.abs(xr), np.abs(wc))
+
+
+# --------------------------------------------------------------------------
+# int8 tied head, last position only
+# --------------------------------------------------------------------------
+
+def dequantize_i8_head(table, scales, K: int, V: int, ldt: int | None = None) -> np.ndarray:
+    """fp32 w[k, v] = q[k, v] * s[v] for the int8 [K, V] table (row stride ldt)."""
+    ldt = V if ldt is None else ldt
+    if ldt < V:
+        raise ValueError("ldt < V")
+    t = np.ascontiguousarray(table, dtype=np.int8).reshape(-1)
+    if t.size < K * ldt - (ldt - V):
+        raise ValueError("table too small")
+    if K == 0 or V == 0:
+        return np.zeros((K, V), np.float32)
+    rows = np.lib.stride_tricks.as_strided(t, shape=(K, V), strides=(ldt, 1))
+    s = np.ascontiguousarray(scales, dtype=np.float32).reshape(V)
+    return rows.astype(np.float32) * s[None, :]  # exact int8 -> fp32, one RN multiply
+
+
+def i8_head_ref(h, table, scales, K: int, V: int, ldt: int | None = None):
+    """Logits of the last-position rows h [M, K]: fp64 (logits, sum|h*w|)."""
+    w = dequantize_i8_head(table, scales, K, V, ldt).astype(np.float64)
+    h64 = _rows(h, K)
+    return h64 @ w, np.abs(h64) @ np.abs(w)
+
+
+def last_position_rows(hidden, T: int, K: int) -> np.ndarray:
+    """Rows T-1 of M sequences of hidden states [M, T, K] (last_token_logits)."""
+    hs = np.asarray(hidden, dtype=np.float32).reshape(-1, T, K)
+    return np.ascontiguousarray(hs[:, T - 1, :])
+
+
+# --------------------------------------------------------------------------
+# tolerance
+# --------------------------------------------------------------------------
+
+def tolerance(a) -> np.ndarray:
+    """Allowed |y - y_ref| per output: 1e-5 * sum|x*w| + 1e-6."""
+    return REL_TOL * np.asarray(a, dtype=np.float64) + ABS_TOL
+
+
+def max_violation(y, y_ref, a) -> float:
+    """max(|y - y_ref| - tol) over outputs; <= 0 means every output passes."""
+    y = np.asarray(y, dtype=np.float64)
+    d = np.abs(y - np.asarray(y_ref, dtype=np.float64)) - tolerance(a)
+    if d.size == 0:
+        return -np.inf
+    if not np.all(np.isfinite(y)):
+        return np.inf
+    return float(d.max())
+
+
+# --------------------------------------------------------------------------
+# quantisers (self-checks of the oracle only; not on the product path)
+# --------------------------------------------------------------------------
+
+def quantize_w4(w) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Asymmetric min/max 4-bit quantiser, per (32-row block, column).
+
+    The page says "asymmetric, blocks of 32 along K" and gives no formula; this
+    is the plainest min/max reading: the range [lo, hi] always contains 0,
+    s = (hi - lo) / 15 stored as fp32, zp = rint(-lo / s) clamped to 0..15,
+    q = rint(w / s) + zp clamped to 0..15 (rint rounds half to even). A block
+    with hi == lo (all zeros) takes s = 1, zp = 0.
+    Returns packed qw, fp32 scales [K/32, N], packed zp.
+    """
+    w = np.asarray(w, dtype=np.float32)
+    K, N = w.shape
+    check_w4_shape(K, N)
+    nb = K // BLOCK
+    wb = w.astype(np.float64).reshape(nb, BLOCK, N)
+    lo = np.minimum(wb.min(axis=1), 0.0)
+    hi = np.maximum(wb.max(axis=1), 0.0)
+    s = ((hi - lo) / 15.0).astype(np.float32)
+    flat = hi == lo
+    s[flat] = 1.0
+    s64 = s.astype(np.float64)
+    zp = np.clip(np.rint(-lo / s64), 0, 15)
+    zp[flat] = 0
+    q = np.clip(np.rint(wb / s64[:, None, :]) + zp[:, None, :], 0, 15)
+    q = q.reshape(K, N).astype(np.uint8)
+    return pack_nibbles(q), s, pack_nibbles(zp.astype(np.uint8))
+
+
+def quantize_i8_head(w) -> tuple[np.ndarray, np.ndarray]:
+    """Symmetric int8 quantiser, one scale per column (token) of [K, V]:
+    s = max|w| / 127, q = rint(w / s) clamped to -127..127; an all-zero
+    column takes s = 1."""
+    w = np.asarray(w, dtype=np.float32)
+    amax = np.abs(w.astype(np.float64)).max(axis=0)
+    s = (amax / 127.0).astype(np.float32)
+    s[amax == 0] = 1.0
+    q = np.clip(np.rint(w.astype(np.float64) / s.astype(np.float64)[None, :]), -127, 127)
+    return q.astype(np.int8), s
