@@ -1,0 +1,447 @@
+"""Throughput of the W4 decode step on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+the 48 W4 body weights of a GPT-2-small-shaped decoder in ONE grouped launch
+(each weight with its own fresh fp32 input row, M = 1), then the int8 tied
+LM head on the last position (M = 1, V = 50257). The metric is effective
+weight GB/s (4-bit nibbles + scales + zero points + int8 table + head scales
+read per step) and decode tokens/s = 1 / step time; the body kernel's GB/s is
+also given as a fraction of the measured HBM copy bandwidth.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs an independent
+replica (the decode step has no cross-GPU exchange); value = all ranks' bytes
+/ the slowest rank's time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes as C
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int8_weight_quantized_w4_b200 import synth  # noqa: E402
+
+METRIC = "weight GB/s and decode tokens/s (GPT-2-small W4 stack, M=1) as % of HBM roofline"
+WORKLOAD = "gpt2-small W4 decode step: 48 body weights (12 x [768x2304, 768x768, 768x3072, 3072x768]) " \
+           "in one grouped launch + int8 tied head [768x50257] on the last position, M=1, fp32"
+HEAD_K, HEAD_V = synth.GPT2_HIDDEN, synth.GPT2_VOCAB
+
+
+def body_bytes() -> int:
+    return sum(synth.w4_bytes(K, N) for _, K, N in synth.gpt2_stack_shapes())
+
+
+def head_bytes() -> int:
+    return synth.i8_head_bytes(HEAD_K, HEAD_V)
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "_source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks
+
+def gpu_id(local: int) -> str:
+    """nvidia-smi id of a torch device (its UUID, whatever CUDA_VISIBLE_DEVICES says)."""
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        return str(local)
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (read-only queries)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, _, parts in rows:
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_init(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- workload
+
+class Workload:
+    """Device-resident weights (R rotating copies), inputs and outputs."""
+
+    def __init__(self, copies: int, seed: int = synth.BASE_SEED):
+        import torch
+        import int8_weight_quantized_w4_b200 as w4
+        self.w4 = w4
+        self.shapes = synth.gpt2_stack_shapes()
+        dev = torch.device("cuda")
+        host_w = [synth.w4_weight(K, N, i, seed=seed) for i, (_, K, N) in enumerate(self.shapes)]
+        H = synth.i8_head(HEAD_K, HEAD_V, seed=seed)
+        self.x_host = [synth.activations(1, K, i, seed=seed) for i, (_, K, _) in enumerate(self.shapes)]
+        self.h_host = synth.activations(1, HEAD_K, 999, seed=seed)
+        self.xs = [torch.from_numpy(x).to(dev) for x in self.x_host]
+        self.h = torch.from_numpy(self.h_host).to(dev)
+        self.ys = [torch.empty((1, N), dtype=torch.float32, device=dev) for _, _, N in self.shapes]
+        self.logits = torch.empty((1, HEAD_V), dtype=torch.float32, device=dev)
+        base = [{k: torch.from_numpy(W[k]).to(dev) for k in ("qw", "scales", "zp")} for W in host_w]
+        table = torch.from_numpy(H["table"]).to(dev)
+        hsc = torch.from_numpy(H["scales"]).to(dev)
+        self.copies = []
+        for r in range(copies):
+            ws = base if r == 0 else [{k: v.clone() for k, v in d.items()} for d in base]
+            items = [{"x": self.xs[i], "y": self.ys[i], "K": K, "N": N, **ws[i]}
+                     for i, (_, K, N) in enumerate(self.shapes)]
+            descs = w4.make_descs(items)
+            t = table if r == 0 else table.clone()
+            s = hsc if r == 0 else hsc.clone()
+            self.copies.append((descs, t, s))
+        need = w4.w4_matmul_grouped_workspace_size(self.copies[0][0])
+        self.ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
+        self.ws_bytes = self.ws.numel()
+        self.lib = w4.lib()
+        torch.cuda.synchronize()
+
+    def body(self, r: int, stream_handle: int):
+        descs = self.copies[r][0]
+        st = self.lib.w4_matmul_grouped(descs, len(descs), self.ws.data_ptr(), self.ws_bytes, stream_handle)
+        if st != 0:
+            raise RuntimeError(f"w4_matmul_grouped failed: {st} {self.lib.w4_last_error()}")
+
+    def head(self, r: int, stream_handle: int):
+        _, t, s = self.copies[r]
+        st = self.lib.i8_head_logits(self.h.data_ptr(), HEAD_K, t.data_ptr(), HEAD_V, s.data_ptr(),
+                                     self.logits.data_ptr(), HEAD_V, 1, HEAD_K, HEAD_V, stream_handle)
+        if st != 0:
+            raise RuntimeError(f"i8_head_logits failed: {st} {self.lib.w4_last_error()}")
+
+
+def rotation_copies(step_bytes: int) -> int:
+    import torch
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    return max(2, -(-3 * l2 // step_bytes) + 1)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    step_bytes = body_bytes() + head_bytes()
+    R = rotation_copies(step_bytes)
+    wl = Workload(R)
+    stream = torch.cuda.current_stream()
+    sh = int(stream.cuda_stream)
+    warm = max(3, args.warmup)
+    for i in range(warm):
+        wl.body(i % R, sh)
+        wl.head(i % R, sh)
+    torch.cuda.synchronize()
+
+    # ---- device-resident timing (value, roofline)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(gpu_id(local if world > 1 else 0))
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.2)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        r = (warm + i) % R
+        ev[i][0].record(stream)
+        wl.body(r, sh)
+        ev[i][1].record(stream)
+        wl.head(r, sh)
+        ev[i][2].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    body_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    head_ms = [b.elapsed_time(c) for _, b, c in ev]
+    ms_step = total_ms / K
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(wl, args, world, R)
+
+    peaks = measured_peaks()
+    body_avg = statistics.mean(body_ms)
+    achieved = body_bytes() / (body_avg * 1e-3) / 1e9
+    n = world
+    value = step_bytes * n / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": n,
+        "steps": K,
+        "warmup": warm,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded uniform nibbles / int8, fp32 N(0,1) activations)",
+        "config": {
+            "workload": WORKLOAD,
+            "weight_bytes_per_step": step_bytes,
+            "body_bytes": body_bytes(),
+            "head_bytes": head_bytes(),
+            "M": 1,
+            "parallelism": f"replicas x{n}" if n > 1 else "1 GPU",
+            "l2": f"rotating {R} weight copies ({R * step_bytes / 1e6:.0f} MB, > 3x L2): every step L2-cold",
+            "seed": synth.BASE_SEED,
+        },
+        "tokens_per_s": round(n * 1e3 / ms_step, 1),
+        "body_only": {"ms": round(body_avg, 5), "GB_per_s": round(achieved, 1),
+                      "tokens_per_s": round(1e3 / body_avg, 1)},
+        "head_only": {"ms": round(statistics.mean(head_ms), 5),
+                      "GB_per_s": round(head_bytes() / (statistics.mean(head_ms) * 1e-3) / 1e9, 1)},
+        "frac_of_hbm_step": round(value / n / peaks["hbm_gbs"], 4),
+        "roofline": {
+            "kernel": "w4_gemv_kernel<1> (grouped 48-weight launch)",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"],
+            "peak_source": f"{peaks['_source']} hbm_gbs (copy, burst)",
+            "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": None,
+        },
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return line
+
+
+def run_e2e(wl, args, world, R):
+    """Same step through the public binding with host buffers: per step, copy
+    the step's inputs from pinned host memory, run body + head, read every
+    output back to pinned host memory."""
+    import torch
+    stream = torch.cuda.current_stream()
+    sh = int(stream.cuda_stream)
+    xh = [torch.from_numpy(x).pin_memory() for x in wl.x_host]
+    hh = torch.from_numpy(wl.h_host).pin_memory()
+    yh = [torch.empty(y.shape, dtype=torch.float32).pin_memory() for y in wl.ys]
+    lh = torch.empty(wl.logits.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(x.numel() * 4 for x in xh) + hh.numel() * 4
+    d2h = sum(y.numel() * 4 for y in yh) + lh.numel() * 4
+
+    def step(r):
+        for d, s in zip(wl.xs, xh):
+            d.copy_(s, non_blocking=True)
+        wl.h.copy_(hh, non_blocking=True)
+        wl.body(r, sh)
+        wl.head(r, sh)
+        for d, s in zip(yh, wl.ys):
+            d.copy_(s, non_blocking=True)
+        lh.copy_(wl.logits, non_blocking=True)
+
+    for i in range(3):
+        step(i % R)
+    torch.cuda.synchronize()
+    K = args.steps
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(K):
+        step(i % R)
+        stream.synchronize()  # the step's result is on the host before the next step
+    el = time.perf_counter() - t0
+    barrier(world)
+    el = max_over_ranks(el, world)
+    step_bytes = body_bytes() + head_bytes()
+    return {"value": round(step_bytes * world / (el / K) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(el / K * 1e3, 5), "tokens_per_s": round(world * K / el, 1)}
+
+
+# ---------------------------------------------------------------- oracle on the host
+
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(budget_s: float) -> dict:
+    """The oracle, as it stands, on this host's cores: whole decode steps of
+    the same workload (48 weights + head), repeated until ~budget_s."""
+    import oracle
+    shapes = synth.gpt2_stack_shapes()
+    ws = [synth.w4_weight(K, N, i) for i, (_, K, N) in enumerate(shapes)]
+    xs = [synth.activations(1, K, i) for i, (_, K, _) in enumerate(shapes)]
+    H = synth.i8_head(HEAD_K, HEAD_V)
+    h = synth.activations(1, HEAD_K, 999)
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        for W, x in zip(ws, xs):
+            oracle.w4_matmul_ref(x, W["qw"], W["scales"], W["zp"], W["K"], W["N"])
+        oracle.i8_head_ref(h, H["table"], H["scales"], HEAD_K, HEAD_V)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or steps >= 50:
+            break
+    per_step = el / steps
+    return {"value": round((body_bytes() + head_bytes()) / per_step / 1e9, 4), "unit": "GB/s",
+            "tokens_per_s": round(1 / per_step, 3), "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{steps} full decode steps (48 weights + head), {el:.1f} s; numpy unpack/dequantize "
+                      f"single-threaded, fp64 matmul on BLAS threads"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    K = args.steps
+    warm = max(0, min(args.warmup, 1))
+    import oracle  # noqa: F401
+    for _ in range(warm):
+        cpu_baseline(0.0)
+    t0 = time.perf_counter()
+    per = []
+    for _ in range(K):
+        s = time.perf_counter()
+        cpu_baseline(0.0)  # exactly one oracle decode step
+        per.append(time.perf_counter() - s)
+    el = time.perf_counter() - t0
+    ms = el / K * 1e3
+    val = (body_bytes() + head_bytes()) / (el / K) / 1e9
+    cb = {"value": round(val, 4), "unit": "GB/s", "cores": _blas_threads(), "kind": "oracle",
+          "sample": f"{K} full decode steps of the same workload on the host"}
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": K, "warmup": warm, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": 1, "weight_bytes_per_step": body_bytes() + head_bytes()},
+            "tokens_per_s": round(1e3 / ms, 3), "cpu_baseline": cb,
+            "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_init(args.gpus)
+    try:
+        line = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

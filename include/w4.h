@@ -1,0 +1,195 @@
+/*
+ * w4.h — C ABI of the B200 quantised-weight matmul library (libw4b200.so).
+ *
+ * Two operations, both fp32 in and out, both hand-written CUDA for sm_100a:
+ *
+ *  w4_matmul       y = x . W, W[K, N] stored 4-bit asymmetric in blocks of 32
+ *                  along K with one fp32 scale and one uint4 zero point per
+ *                  (block, column), dequantised as w = (q - zp) * scale.
+ *                  Source: "ONNX export, quantization and the browser runtime"
+ *                  (tokenling docs), section "Quantization (train/quantize.py)",
+ *                  steps 1 (gemm_to_matmul: plain [K, N] weights, K = in,
+ *                  N = out) and 2 (dq4: 4-bit asymmetric, blocks of 32 along K,
+ *                  fp32 scale + uint4 zero point per block, raw packed UINT4,
+ *                  restored by one blocked DequantizeLinear).
+ *
+ *  i8_head_logits  logits = h . (T * s), T[K, V] int8 with one fp32 scale per
+ *                  token column, applied to the last position only.
+ *                  Source: same page and section, steps 3 (embedding_int8: the
+ *                  tied embedding / LM head stored once as int8, one scale per
+ *                  token, in the head's [768, V] layout) and 4
+ *                  (last_token_logits: the head reads the last position only).
+ *
+ * Data layouts (all row-major):
+ *   x       fp32 [M, K], row stride ldx >= K (elements).
+ *   qw      uint8 [K * N / 2]: element (k, n) of the [K, N] nibble tensor is
+ *           flat index i = k*N + n, stored in byte i >> 1, low nibble when i is
+ *           even ("raw packed UINT4", low nibble first).
+ *   scales  fp32 [K/32, N]; row b holds the scales of rows 32b .. 32b+31.
+ *   zp      uint8 [(K/32) * N / 2]: the [K/32, N] zero-point tensor packed by
+ *           the same rule as qw.
+ *   y       fp32 [M, N], row stride ldy >= N; fully overwritten.
+ *   table   int8 [K, V] with row stride ldt >= V (bytes); row k starts at byte
+ *           k * ldt, which need not be aligned (V = 50257 is odd).
+ *   logits  fp32 [M, V], row stride ldl >= V; fully overwritten.
+ *
+ * Conventions shared by every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller (for example
+ *     torch tensors). The library allocates no device memory and keeps no
+ *     per-call state.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Calls are asynchronous and stream-ordered: nothing inside
+ *     synchronises with the host, except the functions marked SYNCHRONOUS.
+ *   - Every argument check runs before any launch. On failure the call
+ *     returns the status, launches nothing and records a one-line reason that
+ *     w4_last_error() returns on the same host thread.
+ *   - There is no CPU fallback: every result is computed by this library's
+ *     kernels on the GPU, or the call fails.
+ *   - Sizes are int64_t; M = 0 or N = 0 (V = 0) is a valid no-op; K = 0 writes
+ *     zeros (the empty sum).
+ */
+#ifndef W4_B200_H
+#define W4_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define W4_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define W4_API __attribute__((visibility("default")))
+#else
+#define W4_API
+#endif
+
+typedef enum w4_status {
+  W4_OK = 0,
+  W4_ERR_NULL = 1,      /* a required pointer is NULL                                */
+  W4_ERR_SHAPE = 2,     /* K % 32 != 0, N odd, negative size, ld < row length, ...   */
+  W4_ERR_ALIGN = 3,     /* qw / scales / zp not 16-byte aligned; fp32 not 4-byte     */
+  W4_ERR_DEVICE = 4,    /* current device is not sm_100 (B200), or no device          */
+  W4_ERR_CUDA = 5,      /* a CUDA runtime call or launch failed (detail in last_error) */
+  W4_ERR_TIMEOUT = 6,   /* a bounded device-side wait ran out (see w4_device_error)  */
+  W4_ERR_WORKSPACE = 7, /* workspace missing, too small or misaligned                */
+  W4_ERR_VALUE = 8      /* a host-side value out of range (e.g. a nibble > 15)       */
+} w4_status;
+
+/* Kernel choice. W4_PATH_AUTO picks by shape, alignment and M; the others
+ * force one of this library's own kernels (for tests and benchmarks) and
+ * fail with W4_ERR_SHAPE / W4_ERR_ALIGN when that kernel cannot take the
+ * call. */
+typedef enum w4_path {
+  W4_PATH_AUTO = 0,
+  W4_PATH_GEMV = 1,    /* TMA-fed stream-K GEMV: N % 32 == 0, x 16-B aligned, ldx % 4 == 0 */
+  W4_PATH_GENERIC = 2, /* plain-load kernel: any even N, any 4-B aligned x / y                */
+  W4_PATH_TC = 3       /* tcgen05 3xTF32 tile GEMM (large M)                                  */
+} w4_path;
+
+/* One independent matmul of a grouped launch; fields as in w4_matmul. */
+typedef struct w4_desc {
+  const float* x;
+  int64_t ldx;
+  const uint8_t* qw;
+  const float* scales;
+  const uint8_t* zp;
+  float* y;
+  int64_t ldy;
+  int64_t M;
+  int64_t K;
+  int64_t N;
+} w4_desc;
+
+/* ------------------------------------------------------------------ body */
+
+/* Bytes of workspace w4_matmul needs for this shape on the current device
+ * (0 when none is needed). The workspace holds split-K partial sums and one
+ * 32-bit counter per output tile. It must be device memory, 16-byte aligned,
+ * and ZERO-FILLED before its first use; every successful call leaves it
+ * zero-filled again, so one zeroing at allocation suffices. Two calls that
+ * may run at the same time must not share a workspace. After a call that
+ * reported W4_ERR_TIMEOUT, zero it again before reuse. */
+W4_API size_t w4_matmul_workspace_size(int64_t M, int64_t K, int64_t N);
+
+/* y[M, N] = x[M, K] . W[K, N] with W in the 4-bit blocked format above.
+ * Requires K % 32 == 0, N even, ldx >= K, ldy >= N, qw / scales / zp 16-byte
+ * aligned, x / y 4-byte aligned. workspace may be NULL only when
+ * w4_matmul_workspace_size() returns 0. */
+W4_API w4_status w4_matmul(const float* x, int64_t ldx, const uint8_t* qw, const float* scales,
+                    const uint8_t* zp, float* y, int64_t ldy, int64_t M, int64_t K, int64_t N,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* As w4_matmul with an explicit kernel choice. */
+W4_API w4_status w4_matmul_path(const float* x, int64_t ldx, const uint8_t* qw, const float* scales,
+                         const uint8_t* zp, float* y, int64_t ldy, int64_t M, int64_t K,
+                         int64_t N, void* workspace, size_t workspace_bytes, w4_path path,
+                         void* stream);
+
+/* Many independent matmuls (for example the 48 weights of a decoder stack)
+ * in as few launches as possible: up to W4_GROUP_MAX descriptors share one
+ * persistent launch whose work is split evenly over the SMs. `descs` is a
+ * HOST array read during the call only. The outputs must not overlap each
+ * other or any input. */
+#define W4_GROUP_MAX 48
+W4_API size_t w4_matmul_grouped_workspace_size(const w4_desc* descs, int32_t count);
+W4_API w4_status w4_matmul_grouped(const w4_desc* descs, int32_t count, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ head */
+
+/* logits[M, V] = h[M, K] . (T[K, V] * s[V]); the M rows of h are the last
+ * positions of M sequences (pass h = hidden + (T_len - 1) * ldh for one
+ * sequence). Requires ldh >= K, ldt >= V, ldl >= V, h / scales / logits
+ * 4-byte aligned, table 16-byte aligned. No workspace. */
+W4_API w4_status i8_head_logits(const float* h, int64_t ldh, const int8_t* table, int64_t ldt,
+                         const float* scales, float* logits, int64_t ldl, int64_t M, int64_t K,
+                         int64_t V, void* stream);
+
+/* As i8_head_logits with an explicit kernel choice (AUTO, GEMV or GENERIC). */
+W4_API w4_status i8_head_logits_path(const float* h, int64_t ldh, const int8_t* table, int64_t ldt,
+                              const float* scales, float* logits, int64_t ldl, int64_t M,
+                              int64_t K, int64_t V, w4_path path, void* stream);
+
+/* ------------------------------------------------------------------ host packing */
+
+/* Pack n uint4 values (each 0..15) into (n + 1) / 2 bytes, low nibble first;
+ * an odd n leaves the last high nibble 0. Host memory. W4_ERR_VALUE if a
+ * value exceeds 15 (nothing is written then). */
+W4_API w4_status w4_pack_nibbles(const uint8_t* q, int64_t n, uint8_t* out);
+
+/* Unpack the first n nibbles of `packed` (host memory) into q[n]. */
+W4_API w4_status w4_unpack_nibbles(const uint8_t* packed, int64_t n, uint8_t* q);
+
+/* ------------------------------------------------------------------ diagnostics */
+
+W4_API const char* w4_status_string(w4_status s);
+
+/* One-line reason for the last non-OK status returned on this host thread. */
+W4_API const char* w4_last_error(void);
+
+/* SYNCHRONOUS. Reads the current device's error word, which a kernel sets
+ * when one of its bounded waits runs out (kernels never trap, assert or spin
+ * without limit). info (may be NULL) receives {status, kernel id, block
+ * index, detail}. With clear != 0 the word is reset to 0. Returns the
+ * recorded status (W4_OK if none) or W4_ERR_CUDA if the read itself failed. */
+W4_API w4_status w4_device_error(int32_t* info4, int32_t clear);
+
+/* Limit of every bounded device wait, in nanoseconds (default 2e9). */
+W4_API w4_status w4_set_wait_timeout_ns(uint64_t ns);
+
+/* Launches a kernel that waits, through the same bounded-wait code the
+ * matmul kernels use, on a barrier nothing ever completes, with the given
+ * limit. It records W4_ERR_TIMEOUT in the device error word and returns;
+ * used to test the timeout path without hanging a GPU. */
+W4_API w4_status w4_debug_wait_timeout(uint64_t timeout_ns, void* stream);
+
+W4_API int32_t w4_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4_B200_H */

@@ -1,0 +1,198 @@
+"""B200 quantised-weight matmul library: Python binding of libw4b200.so.
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels (sm_100a). PyTorch provides device memory and
+streams. If the library is missing or the GPU is not a B200 the calls raise;
+nothing falls back to another implementation.
+
+Operations (see include/w4.h for layouts and error behaviour):
+  w4_matmul(x, qw, scales, zp, K, N)        y = x . W, W 4-bit blocked
+  w4_matmul_grouped([...])                  many independent ones, one launch
+  i8_head_logits(h, table, scales, K, V)    last-position logits, int8 head
+  pack_nibbles / unpack_nibbles             host-side UINT4 packing
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+from typing import Sequence
+
+import numpy as np
+
+from . import _lib
+from ._lib import GROUP_MAX, PATHS, STATUS, W4Desc, W4LibraryMissing  # noqa: F401
+
+
+class W4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        detail = ""
+        try:
+            detail = (_lib.load().w4_last_error() or b"").decode()
+        except Exception:
+            pass
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {detail}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise W4Error(status, where)
+
+
+def lib():
+    return _lib.load()
+
+
+def abi_version() -> int:
+    return lib().w4_abi_version()
+
+
+# ---------------------------------------------------------------- torch helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _stream_handle(stream) -> int:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+_WS = {}  # device index -> zero-filled uint8 workspace tensor
+
+
+def workspace(nbytes: int, device=None):
+    """A zero-filled device workspace of at least nbytes (cached per device).
+
+    The kernels leave it zero-filled, so it is zeroed only when allocated.
+    Calls that may overlap on the GPU must not share one: pass your own.
+    """
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    idx = dev.index if dev.index is not None else torch.cuda.current_device()
+    cur = _WS.get(idx)
+    if nbytes == 0:
+        return None
+    if cur is None or cur.numel() < nbytes:
+        cur = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=dev)
+        _WS[idx] = cur
+    return cur
+
+
+def _ld(t, inner: int) -> int:
+    if t.dim() == 1:
+        return inner
+    if t.stride(-1) != 1:
+        raise ValueError("innermost dimension must be contiguous")
+    return int(t.stride(0))
+
+
+# ---------------------------------------------------------------- body
+
+def w4_matmul_workspace_size(M: int, K: int, N: int) -> int:
+    return int(lib().w4_matmul_workspace_size(M, K, N))
+
+
+def w4_matmul(x, qw, scales, zp, K: int, N: int, y=None, path: str = "auto", ws=None, stream=None):
+    """y[M, N] = x[M, K] . W[K, N] (fp32) with W given as packed nibbles,
+    fp32 scales [K/32, N] and packed zero points; returns y."""
+    torch = _torch()
+    M = x.shape[0] if x.dim() == 2 else 1
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    need = w4_matmul_workspace_size(M, K, N)
+    if ws is None:
+        ws = workspace(need, x.device)
+    st = lib().w4_matmul_path(_ptr(x), _ld(x, K), _ptr(qw), _ptr(scales), _ptr(zp), _ptr(y), _ld(y, N), M, K, N,
+                              _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), PATHS[path],
+                              _stream_handle(stream))
+    _check(st, "w4_matmul")
+    return y
+
+
+def make_descs(items: Sequence[dict]):
+    """ctypes descriptor array for w4_matmul_grouped; each item holds the
+    tensors x, qw, scales, zp, y and the ints K, N (M from x)."""
+    arr = (W4Desc * len(items))()
+    for i, it in enumerate(items):
+        x, y = it["x"], it["y"]
+        K, N = int(it["K"]), int(it["N"])
+        M = x.shape[0] if x.dim() == 2 else 1
+        arr[i] = W4Desc(_ptr(x), _ld(x, K), _ptr(it["qw"]), _ptr(it["scales"]), _ptr(it["zp"]), _ptr(y),
+                        _ld(y, N), M, K, N)
+    return arr
+
+
+def w4_matmul_grouped_workspace_size(descs) -> int:
+    return int(lib().w4_matmul_grouped_workspace_size(descs, len(descs)))
+
+
+def w4_matmul_grouped(items: Sequence[dict] | None = None, descs=None, ws=None, stream=None):
+    """All matmuls of `items` (or a prepared descriptor array) in grouped launches."""
+    if descs is None:
+        descs = make_descs(items)
+    need = w4_matmul_grouped_workspace_size(descs)
+    if ws is None:
+        ws = workspace(need)
+    st = lib().w4_matmul_grouped(descs, len(descs), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                 _stream_handle(stream))
+    _check(st, "w4_matmul_grouped")
+
+
+# ---------------------------------------------------------------- head
+
+def i8_head_logits(h, table, scales, K: int, V: int, ldt: int | None = None, logits=None, path: str = "auto",
+                   stream=None):
+    """logits[M, V] = h[M, K] . (T[K, V] * s[V]) for the int8 tied head; h holds
+    the last-position rows."""
+    torch = _torch()
+    M = h.shape[0] if h.dim() == 2 else 1
+    ldt = V if ldt is None else ldt
+    if logits is None:
+        logits = torch.empty((M, V), dtype=torch.float32, device=h.device)
+    st = lib().i8_head_logits_path(_ptr(h), _ld(h, K), _ptr(table), ldt, _ptr(scales), _ptr(logits),
+                                   _ld(logits, V), M, K, V, PATHS[path], _stream_handle(stream))
+    _check(st, "i8_head_logits")
+    return logits
+
+
+# ---------------------------------------------------------------- host packing
+
+def pack_nibbles(q) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8).reshape(-1)
+    out = np.zeros((q.size + 1) // 2, dtype=np.uint8)
+    _check(lib().w4_pack_nibbles(q.ctypes.data, q.size, out.ctypes.data), "w4_pack_nibbles")
+    return out
+
+
+def unpack_nibbles(packed, n: int) -> np.ndarray:
+    p = np.ascontiguousarray(packed, dtype=np.uint8).reshape(-1)
+    if 2 * p.size < n:
+        raise ValueError("buffer too small")
+    out = np.zeros(n, dtype=np.uint8)
+    _check(lib().w4_unpack_nibbles(p.ctypes.data, n, out.ctypes.data), "w4_unpack_nibbles")
+    return out
+
+
+# ---------------------------------------------------------------- diagnostics
+
+def device_error(clear: bool = True):
+    """(status, [status, kernel, block, detail]) of the current device's error word."""
+    info = (C.c_int32 * 4)()
+    st = lib().w4_device_error(info, 1 if clear else 0)
+    return st, list(info)
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    _check(lib().w4_set_wait_timeout_ns(ns), "w4_set_wait_timeout_ns")
+
+
+def debug_wait_timeout(ns: int, stream=None) -> None:
+    _check(lib().w4_debug_wait_timeout(ns, _stream_handle(stream)), "w4_debug_wait_timeout")

@@ -1,0 +1,360 @@
+// extern "C" boundary of libw4b200: argument checks, kernel choice, device
+// properties, tensor-map encoding, host-side nibble packing, diagnostics.
+// Every check runs before any launch; a failed check launches nothing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+
+#include "w4_device.cuh"
+#include "w4_internal.h"
+
+// One error word per device that loads the library (see w4_device_error).
+__device__ w4dev::ErrorWord g_w4_error_word;
+
+namespace w4host {
+
+namespace {
+
+thread_local char t_detail[512] = "";
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+constexpr int kMaxDev = 64;
+DeviceInfo g_dev[kMaxDev];
+std::once_flag g_dev_once[kMaxDev];
+w4_status g_dev_status[kMaxDev];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void init_device(int dev) {
+  DeviceInfo& d = g_dev[dev];
+  d.dev = dev;
+  cudaDeviceProp prop;
+  cudaError_t e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) {
+    g_dev_status[dev] = W4_ERR_CUDA;
+    return;
+  }
+  d.sms = prop.multiProcessorCount;
+  d.major = prop.major;
+  d.minor = prop.minor;
+  d.smem_optin = prop.sharedMemPerBlockOptin;
+  if (!(prop.major == 10 && prop.minor == 0)) {
+    g_dev_status[dev] = W4_ERR_DEVICE;
+    return;
+  }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_w4_error_word);
+  if (e != cudaSuccess) {
+    g_dev_status[dev] = W4_ERR_CUDA;
+    return;
+  }
+  d.err = static_cast<w4dev::ErrorWord*>(p);
+  g_dev_status[dev] = W4_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace
+
+w4_status fail(w4_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_detail, sizeof(t_detail), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+w4_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(W4_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+uint64_t wait_timeout_ns() { return g_timeout_ns.load(std::memory_order_relaxed); }
+
+w4_status current_device(const DeviceInfo** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(W4_ERR_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDev) return fail(W4_ERR_DEVICE, "device index %d out of range", dev);
+  std::call_once(g_dev_once[dev], init_device, dev);
+  if (g_dev_status[dev] == W4_ERR_DEVICE)
+    return fail(W4_ERR_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a (B200) only", dev,
+                g_dev[dev].major, g_dev[dev].minor);
+  if (g_dev_status[dev] != W4_OK) return fail(g_dev_status[dev], "device %d could not be queried", dev);
+  *out = &g_dev[dev];
+  return W4_OK;
+}
+
+w4_status encode_qw_map(CUtensorMap* map, const uint8_t* qw, int64_t K, int64_t N) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (g_encode == nullptr) return fail(W4_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N / 2), static_cast<cuuint64_t>(K)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N / 2)};
+  const cuuint32_t box[2] = {128, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(qw), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for K=%lld N=%lld", int(r),
+                                     (long long)K, (long long)N);
+  return W4_OK;
+}
+
+// ------------------------------------------------------------------ validation
+
+static w4_status check_desc(const w4_desc& d) {
+  if (d.M < 0 || d.K < 0 || d.N < 0) return fail(W4_ERR_SHAPE, "negative size (M=%lld K=%lld N=%lld)",
+                                                 (long long)d.M, (long long)d.K, (long long)d.N);
+  if (d.K % 32 != 0) return fail(W4_ERR_SHAPE, "K=%lld is not a multiple of 32", (long long)d.K);
+  if (d.N % 2 != 0) return fail(W4_ERR_SHAPE, "N=%lld is odd", (long long)d.N);
+  if (d.M == 0 || d.N == 0) return W4_OK;
+  if (d.y == nullptr) return fail(W4_ERR_NULL, "y is NULL");
+  if (d.ldy < d.N) return fail(W4_ERR_SHAPE, "ldy=%lld < N=%lld", (long long)d.ldy, (long long)d.N);
+  if (!aligned(d.y, 4)) return fail(W4_ERR_ALIGN, "y must be 4-byte aligned");
+  if (d.K == 0) return W4_OK;
+  if (d.x == nullptr || d.qw == nullptr || d.scales == nullptr || d.zp == nullptr)
+    return fail(W4_ERR_NULL, "x, qw, scales and zp must not be NULL");
+  if (d.ldx < d.K) return fail(W4_ERR_SHAPE, "ldx=%lld < K=%lld", (long long)d.ldx, (long long)d.K);
+  if (!aligned(d.qw, 16) || !aligned(d.scales, 16) || !aligned(d.zp, 16))
+    return fail(W4_ERR_ALIGN, "qw, scales and zp must be 16-byte aligned");
+  if (!aligned(d.x, 4)) return fail(W4_ERR_ALIGN, "x must be 4-byte aligned");
+  return W4_OK;
+}
+
+}  // namespace w4host
+
+using namespace w4host;
+
+extern "C" {
+
+int32_t w4_abi_version(void) { return W4_ABI_VERSION; }
+
+const char* w4_status_string(w4_status s) {
+  switch (s) {
+    case W4_OK: return "W4_OK";
+    case W4_ERR_NULL: return "W4_ERR_NULL";
+    case W4_ERR_SHAPE: return "W4_ERR_SHAPE";
+    case W4_ERR_ALIGN: return "W4_ERR_ALIGN";
+    case W4_ERR_DEVICE: return "W4_ERR_DEVICE";
+    case W4_ERR_CUDA: return "W4_ERR_CUDA";
+    case W4_ERR_TIMEOUT: return "W4_ERR_TIMEOUT";
+    case W4_ERR_WORKSPACE: return "W4_ERR_WORKSPACE";
+    case W4_ERR_VALUE: return "W4_ERR_VALUE";
+  }
+  return "W4_ERR_UNKNOWN";
+}
+
+const char* w4_last_error(void) { return t_detail; }
+
+w4_status w4_set_wait_timeout_ns(uint64_t ns) {
+  if (ns == 0) return fail(W4_ERR_VALUE, "timeout must be positive");
+  g_timeout_ns.store(ns);
+  return W4_OK;
+}
+
+// ------------------------------------------------------------------ packing
+
+w4_status w4_pack_nibbles(const uint8_t* q, int64_t n, uint8_t* out) {
+  if (n < 0) return fail(W4_ERR_SHAPE, "negative count");
+  if (n == 0) return W4_OK;
+  if (q == nullptr || out == nullptr) return fail(W4_ERR_NULL, "NULL buffer");
+  for (int64_t i = 0; i < n; ++i)
+    if (q[i] > 15) return fail(W4_ERR_VALUE, "value %u at %lld exceeds 15", unsigned(q[i]), (long long)i);
+  for (int64_t i = 0; i + 1 < n; i += 2) out[i / 2] = static_cast<uint8_t>(q[i] | (q[i + 1] << 4));
+  if (n & 1) out[n / 2] = q[n - 1];
+  return W4_OK;
+}
+
+w4_status w4_unpack_nibbles(const uint8_t* packed, int64_t n, uint8_t* q) {
+  if (n < 0) return fail(W4_ERR_SHAPE, "negative count");
+  if (n == 0) return W4_OK;
+  if (q == nullptr || packed == nullptr) return fail(W4_ERR_NULL, "NULL buffer");
+  for (int64_t i = 0; i < n; ++i) q[i] = (i & 1) ? (packed[i / 2] >> 4) : (packed[i / 2] & 0x0F);
+  return W4_OK;
+}
+
+// ------------------------------------------------------------------ body
+
+size_t w4_matmul_workspace_size(int64_t M, int64_t K, int64_t N) {
+  const DeviceInfo* di = nullptr;
+  if (current_device(&di) != W4_OK || M <= 0 || K <= 0 || N <= 0 || K % 32 || N % 2) return 0;
+  w4_desc d = {};
+  d.M = M;
+  d.K = K;
+  d.N = N;
+  return gemv_workspace_bytes(&d, 1, di->sms);
+}
+
+static w4_status matmul_one(const w4_desc& d, void* ws, size_t wsb, w4_path path, cudaStream_t st) {
+  w4_status rc = check_desc(d);
+  if (rc != W4_OK) return rc;
+  if (path < W4_PATH_AUTO || path > W4_PATH_TC) return fail(W4_ERR_VALUE, "unknown path %d", int(path));
+  if (d.M == 0 || d.N == 0) return W4_OK;
+  const DeviceInfo* di = nullptr;
+  rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  if (d.K == 0) return launch_zero_fill(d.y, d.ldy, d.M, d.N, st);
+  const char* why = "";
+  const bool gemv_ok = gemv_eligible(d, &why);
+  switch (path) {
+    case W4_PATH_GENERIC: return launch_generic(d, st, *di);
+    case W4_PATH_GEMV:
+      if (!gemv_ok) return fail(W4_ERR_ALIGN, "%s", why);
+      return launch_gemv(&d, 1, ws, wsb, st, *di);
+    case W4_PATH_TC: return fail(W4_ERR_SHAPE, "the tcgen05 path is not available in this build");
+    default:
+      return gemv_ok ? launch_gemv(&d, 1, ws, wsb, st, *di) : launch_generic(d, st, *di);
+  }
+}
+
+w4_status w4_matmul_path(const float* x, int64_t ldx, const uint8_t* qw, const float* scales, const uint8_t* zp,
+                         float* y, int64_t ldy, int64_t M, int64_t K, int64_t N, void* workspace,
+                         size_t workspace_bytes, w4_path path, void* stream) {
+  const w4_desc d = {x, ldx, qw, scales, zp, y, ldy, M, K, N};
+  return matmul_one(d, workspace, workspace_bytes, path, static_cast<cudaStream_t>(stream));
+}
+
+w4_status w4_matmul(const float* x, int64_t ldx, const uint8_t* qw, const float* scales, const uint8_t* zp, float* y,
+                    int64_t ldy, int64_t M, int64_t K, int64_t N, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  return w4_matmul_path(x, ldx, qw, scales, zp, y, ldy, M, K, N, workspace, workspace_bytes, W4_PATH_AUTO, stream);
+}
+
+size_t w4_matmul_grouped_workspace_size(const w4_desc* descs, int32_t count) {
+  const DeviceInfo* di = nullptr;
+  if (descs == nullptr || count <= 0 || current_device(&di) != W4_OK) return 0;
+  size_t best = 0;
+  for (int32_t i = 0; i < count; i += W4_GROUP_MAX) {
+    const int32_t n = count - i < W4_GROUP_MAX ? count - i : W4_GROUP_MAX;
+    const size_t b = gemv_workspace_bytes(descs + i, n, di->sms);
+    best = b > best ? b : best;
+  }
+  return best;
+}
+
+w4_status w4_matmul_grouped(const w4_desc* descs, int32_t count, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (count < 0) return fail(W4_ERR_SHAPE, "negative count");
+  if (count == 0) return W4_OK;
+  if (descs == nullptr) return fail(W4_ERR_NULL, "descs is NULL");
+  for (int32_t i = 0; i < count; ++i) {
+    const w4_status rc = check_desc(descs[i]);
+    if (rc != W4_OK) {
+      char why[sizeof(t_detail)];
+      snprintf(why, sizeof(why), "%s", t_detail);
+      return fail(rc, "descriptor %d: %s", i, why);
+    }
+  }
+  const DeviceInfo* di = nullptr;
+  w4_status rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Split: descriptors the GEMV can take go into grouped launches; the rest
+  // (K = 0, odd layouts) run one by one on their own kernels.
+  static thread_local w4_desc fast[W4_GROUP_MAX];
+  int nfast = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    const w4_desc& d = descs[i];
+    if (d.M == 0 || d.N == 0) continue;
+    const char* why = "";
+    if (d.K == 0) {
+      rc = launch_zero_fill(d.y, d.ldy, d.M, d.N, st);
+    } else if (!gemv_eligible(d, &why)) {
+      rc = launch_generic(d, st, *di);
+    } else {
+      fast[nfast++] = d;
+      if (nfast == W4_GROUP_MAX) {
+        rc = launch_gemv(fast, nfast, workspace, workspace_bytes, st, *di);
+        nfast = 0;
+      }
+    }
+    if (rc != W4_OK) return rc;
+  }
+  if (nfast > 0) rc = launch_gemv(fast, nfast, workspace, workspace_bytes, st, *di);
+  return rc;
+}
+
+// ------------------------------------------------------------------ head
+
+static w4_status head_impl(const HeadArgs& a, w4_path path, cudaStream_t st) {
+  if (a.M < 0 || a.K < 0 || a.V < 0) return fail(W4_ERR_SHAPE, "negative size");
+  if (path != W4_PATH_AUTO && path != W4_PATH_GEMV && path != W4_PATH_GENERIC)
+    return fail(W4_ERR_VALUE, "path %d is not a head path", int(path));
+  if (a.M == 0 || a.V == 0) return W4_OK;
+  if (a.logits == nullptr) return fail(W4_ERR_NULL, "logits is NULL");
+  if (a.ldl < a.V) return fail(W4_ERR_SHAPE, "ldl < V");
+  if (!aligned(a.logits, 4)) return fail(W4_ERR_ALIGN, "logits must be 4-byte aligned");
+  if (a.K > 0) {
+    if (a.h == nullptr || a.table == nullptr || a.scales == nullptr)
+      return fail(W4_ERR_NULL, "h, table and scales must not be NULL");
+    if (a.ldh < a.K) return fail(W4_ERR_SHAPE, "ldh < K");
+    if (a.ldt < a.V) return fail(W4_ERR_SHAPE, "ldt < V");
+    if (!aligned(a.h, 4) || !aligned(a.scales, 4)) return fail(W4_ERR_ALIGN, "h and scales must be 4-byte aligned");
+    if (!aligned(a.table, 16)) return fail(W4_ERR_ALIGN, "table must be 16-byte aligned");
+  }
+  const DeviceInfo* di = nullptr;
+  w4_status rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  if (a.K == 0) return launch_zero_fill(a.logits, a.ldl, a.M, a.V, st);
+  if (path == W4_PATH_GENERIC) return launch_head_generic(a, st, *di);
+  return launch_head(a, st, *di);
+}
+
+w4_status i8_head_logits_path(const float* h, int64_t ldh, const int8_t* table, int64_t ldt, const float* scales,
+                              float* logits, int64_t ldl, int64_t M, int64_t K, int64_t V, w4_path path,
+                              void* stream) {
+  const HeadArgs a = {h, ldh, table, ldt, scales, logits, ldl, M, K, V};
+  return head_impl(a, path, static_cast<cudaStream_t>(stream));
+}
+
+w4_status i8_head_logits(const float* h, int64_t ldh, const int8_t* table, int64_t ldt, const float* scales,
+                         float* logits, int64_t ldl, int64_t M, int64_t K, int64_t V, void* stream) {
+  return i8_head_logits_path(h, ldh, table, ldt, scales, logits, ldl, M, K, V, W4_PATH_AUTO, stream);
+}
+
+// ------------------------------------------------------------------ diagnostics
+
+w4_status w4_device_error(int32_t* info4, int32_t clear) {
+  const DeviceInfo* di = nullptr;
+  w4_status rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  w4dev::ErrorWord w = {};
+  cudaError_t e = cudaMemcpyFromSymbol(&w, g_w4_error_word, sizeof(w));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (info4 != nullptr) {
+    info4[0] = w.status;
+    info4[1] = w.kernel;
+    info4[2] = w.block;
+    info4[3] = w.detail;
+  }
+  if (clear) {
+    const w4dev::ErrorWord z = {};
+    e = cudaMemcpyToSymbol(g_w4_error_word, &z, sizeof(z));
+    if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  }
+  return static_cast<w4_status>(w.status);
+}
+
+w4_status w4_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
+  const DeviceInfo* di = nullptr;
+  w4_status rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return fail(W4_ERR_VALUE, "timeout must be in (0, 10 s]");
+  return launch_debug_wait(timeout_ns, static_cast<cudaStream_t>(stream), *di);
+}
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+// Device-side helpers shared by the kernels of libw4b200: shared-memory
+// barriers, bounded waits, bulk / tensor copies, the nibble decoder.
+//
+// Every wait on a barrier is bounded by %globaltimer: when the limit runs
+// out the waiting thread records W4_ERR_TIMEOUT in the device error word and
+// reports failure to its caller, which stops issuing work and returns. No
+// kernel here traps, asserts or spins without limit.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+#include "w4.h"
+
+namespace w4dev {
+
+// Device error word: {status, kernel id, block index, detail}. Only the first
+// error is kept (compare-and-swap on the status slot).
+struct ErrorWord {
+  int32_t status;
+  int32_t kernel;
+  int32_t block;
+  int32_t detail;
+};
+
+enum KernelId : int32_t { K_GEMV = 1, K_GENERIC = 2, K_HEAD = 3, K_HEAD_GENERIC = 4, K_TC = 5, K_DEBUG = 9 };
+
+__device__ __forceinline__ void record_error(ErrorWord* e, int32_t status, int32_t kernel, int32_t detail) {
+  if (atomicCAS(&e->status, 0, status) == 0) {
+    e->kernel = kernel;
+    e->block = static_cast<int32_t>(blockIdx.x);
+    e->detail = detail;
+    __threadfence();
+  }
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait until the phase with parity `parity` of `bar` has completed. Returns
+// false (after recording the error) when `timeout_ns` passes first, or at
+// once when *abort is already set by another thread of the CTA.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
+                                                  volatile int* abort, ErrorWord* err, int32_t kernel,
+                                                  int32_t detail) {
+  const uint32_t a = smem_u32(bar);
+#pragma unroll 1
+  for (int i = 0; i < 32; ++i)
+    if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
+  while (true) {
+    if (mbar_try_wait(a, parity)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      if (abort != nullptr) *abort = 1;
+      record_error(err, W4_ERR_TIMEOUT, kernel, detail);
+      return false;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- bulk copies (no multicast)
+
+// Untiled bulk copy global -> this CTA's shared memory; completes `bytes`
+// transaction bytes on `bar`. Both addresses 16-B aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 2-D tiled tensor copy global -> this CTA's shared memory (box from map).
+// c0 is the innermost coordinate in elements (bytes for uint8 maps) and must
+// be a multiple of 16 bytes; c1 any row index (rows past the end read zeros).
+__device__ __forceinline__ void tma_g2s_2d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c1,
+                                           uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------- named barriers
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------- nibble decode
+//
+// A 32-bit word holds 8 nibbles n0..n7 (n_i in bits 4i..4i+3). For i in 0..3
+// the float with bits 0x4B000000 | (word & (0xF << 4i)) equals 2^23 + n_i*16^i
+// exactly (the nibble lands inside the 23-bit mantissa of 2^23); for i in
+// 4..7 the same holds on word >> 16 with 16^(i-4). Subtracting the float
+// built the same way from the zero-point word gives (q - zp) * 16^(i mod 4)
+// exactly: both operands are integers in [2^23, 2^24). The power of two is
+// folded into the scale, s * 16^-(i mod 4), which is exact too.
+
+__device__ __forceinline__ float magic_nib(uint32_t word, int slot /*0..3*/) {
+  return __uint_as_float(0x4B000000u | (word & (0xFu << (4 * slot))));
+}
+
+__device__ __forceinline__ float inv_slot_scale(int slot) {
+  return slot == 0 ? 1.0f : (slot == 1 ? 0.0625f : (slot == 2 ? 0.00390625f : 0.000244140625f));
+}
+
+}  // namespace w4dev

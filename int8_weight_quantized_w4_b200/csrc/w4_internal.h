@@ -1,0 +1,64 @@
+// Host-side internals of libw4b200 shared between its translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+#include <cstring>
+
+#include "w4.h"
+
+namespace w4dev {
+struct ErrorWord;
+}
+
+namespace w4host {
+
+struct DeviceInfo {
+  int dev = -1;
+  int sms = 0;
+  int major = 0;
+  int minor = 0;
+  size_t smem_optin = 0;
+  w4dev::ErrorWord* err = nullptr;  // device address of this device's error word
+};
+
+// Current device's cached properties (W4_ERR_DEVICE unless it is sm_100).
+w4_status current_device(const DeviceInfo** out);
+
+// Record a one-line reason for the calling thread and return `s`.
+w4_status fail(w4_status s, const char* fmt, ...);
+w4_status cuda_fail(cudaError_t e, const char* what);
+uint64_t wait_timeout_ns();
+
+// Tensor map of a [K rows][N/2 bytes] nibble matrix, box 32 rows x 128 bytes.
+w4_status encode_qw_map(CUtensorMap* map, const uint8_t* qw, int64_t K, int64_t N);
+
+// ---- body kernels
+bool gemv_eligible(const w4_desc& d, const char** why);
+size_t gemv_workspace_bytes(const w4_desc* d, int count, int sms);
+w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cudaStream_t st,
+                      const DeviceInfo& di);
+w4_status launch_generic(const w4_desc& d, cudaStream_t st, const DeviceInfo& di);
+w4_status launch_zero_fill(float* y, int64_t ldy, int64_t M, int64_t N, cudaStream_t st);
+
+// ---- head kernels
+struct HeadArgs {
+  const float* h;
+  int64_t ldh;
+  const int8_t* table;
+  int64_t ldt;
+  const float* scales;
+  float* logits;
+  int64_t ldl;
+  int64_t M, K, V;
+};
+w4_status launch_head(const HeadArgs& a, cudaStream_t st, const DeviceInfo& di);
+w4_status launch_head_generic(const HeadArgs& a, cudaStream_t st, const DeviceInfo& di);
+
+// ---- diagnostics
+w4_status launch_debug_wait(uint64_t timeout_ns, cudaStream_t st, const DeviceInfo& di);
+
+}  // namespace w4host

@@ -1,0 +1,130 @@
+"""The C-ABI library loads, exports what include/w4.h declares, and refuses bad
+arguments before touching a device (CPU only: no compute calls here)."""
+
+import ctypes as C
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4.h")
+
+
+def _lib():
+    from int8_weight_quantized_w4_b200 import _lib as L
+    if not os.path.exists(L.LIB_PATH):
+        from int8_weight_quantized_w4_b200 import build
+        build.build(quiet=True)
+    return L.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^W4_API\s+[\w\s\*]+?\b(\w+)\(", src, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("w4_matmul", "i8_head_logits", "w4_matmul_grouped", "w4_pack_nibbles", "w4_unpack_nibbles",
+                 "w4_status_string", "w4_device_error"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib()
+    from int8_weight_quantized_w4_b200 import _lib as L
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (\w+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+        assert name in L.SIGNATURES, f"binding lacks {name}"
+
+
+def test_abi_version_and_status_strings():
+    lib = _lib()
+    assert lib.w4_abi_version() == 1
+    assert lib.w4_status_string(0) == b"W4_OK"
+    assert lib.w4_status_string(6) == b"W4_ERR_TIMEOUT"
+    assert lib.w4_status_string(99) == b"W4_ERR_UNKNOWN"
+
+
+def test_host_pack_unpack_exhaustive_against_oracle():
+    from int8_weight_quantized_w4_b200 import pack_nibbles, unpack_nibbles
+    allb = np.arange(256, dtype=np.uint8)
+    assert np.array_equal(unpack_nibbles(allb, 512), oracle.unpack_nibbles(allb, 512))
+    pairs = np.array([(lo, hi) for hi in range(16) for lo in range(16)], np.uint8).reshape(-1)
+    assert np.array_equal(pack_nibbles(pairs), oracle.pack_nibbles(pairs))
+    odd = np.arange(15, dtype=np.uint8)
+    assert np.array_equal(pack_nibbles(odd), oracle.pack_nibbles(odd))
+    assert list(unpack_nibbles(np.array([0x21], np.uint8), 2)) == [1, 2]
+
+
+def test_host_pack_rejects_values_above_15():
+    from int8_weight_quantized_w4_b200 import W4Error, pack_nibbles
+    with pytest.raises(W4Error) as e:
+        pack_nibbles(np.array([1, 16], np.uint8))
+    assert e.value.status == 8
+
+
+def _matmul(lib, x=0x1000, ldx=64, qw=0x2000, sc=0x3000, zp=0x4000, y=0x5000, ldy=64, M=1, K=64, N=64,
+            path=0):
+    return lib.w4_matmul_path(x, ldx, qw, sc, zp, y, ldy, M, K, N, None, 0, path, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=33), 2), (dict(K=-32), 2), (dict(N=63), 2), (dict(M=-1), 2),
+    (dict(ldx=32), 2), (dict(ldy=32), 2),
+    (dict(y=0), 1), (dict(qw=0), 1), (dict(x=0), 1), (dict(zp=0), 1), (dict(sc=0), 1),
+    (dict(qw=0x2008), 3), (dict(sc=0x3004), 3), (dict(zp=0x4001), 3), (dict(x=0x1002), 3), (dict(y=0x5001), 3),
+    (dict(path=7), 8),
+])
+def test_matmul_argument_errors_before_any_launch(kw, status):
+    lib = _lib()
+    assert _matmul(lib, **kw) == status
+    assert lib.w4_last_error()  # a reason is recorded
+
+
+def test_matmul_noops_need_no_device():
+    lib = _lib()
+    assert _matmul(lib, M=0) == 0
+    assert _matmul(lib, N=0) == 0
+    assert _matmul(lib, M=0, x=0, qw=0, sc=0, zp=0, y=0) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=-1), 2), (dict(ldl=10), 2), (dict(ldt=10), 2), (dict(ldh=10), 2),
+    (dict(table=0x2001), 3), (dict(h=0x1002), 3), (dict(logits=0), 1), (dict(table=0), 1),
+])
+def test_head_argument_errors(kw, status):
+    lib = _lib()
+    a = dict(h=0x1000, ldh=32, table=0x2000, ldt=20, scales=0x3000, logits=0x4000, ldl=20, M=1, K=32, V=20)
+    a.update(kw)
+    st = lib.i8_head_logits(a["h"], a["ldh"], a["table"], a["ldt"], a["scales"], a["logits"], a["ldl"], a["M"],
+                            a["K"], a["V"], None)
+    assert st == status
+
+
+def test_grouped_argument_errors():
+    lib = _lib()
+    from int8_weight_quantized_w4_b200._lib import W4Desc
+    d = (W4Desc * 2)()
+    d[0] = W4Desc(0x1000, 64, 0x2000, 0x3000, 0x4000, 0x5000, 64, 1, 64, 64)
+    d[1] = W4Desc(0x1000, 64, 0x2000, 0x3000, 0x4000, 0x5000, 64, 1, 40, 64)
+    assert lib.w4_matmul_grouped(d, 2, None, 0, None) == 2
+    assert b"descriptor 1" in lib.w4_last_error()
+    assert lib.w4_matmul_grouped(d, 0, None, 0, None) == 0
+    assert lib.w4_matmul_grouped(None, 3, None, 0, None) == 1
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    from int8_weight_quantized_w4_b200 import _lib as L
+    monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(L, "_lib", None)
+    with pytest.raises(L.W4LibraryMissing):
+        L.load()
