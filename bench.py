@@ -185,8 +185,10 @@ class Workload:
             descs = w4.make_descs(items)
             t = table if r == 0 else table.clone()
             s = hsc if r == 0 else hsc.clone()
-            self.copies.append((descs, t, s))
-        need = w4.w4_matmul_grouped_workspace_size(self.copies[0][0])
+            # the descriptors hold raw pointers: keep every tensor they name alive
+            self.copies.append((descs, t, s, ws))
+        need = max(w4.w4_matmul_grouped_workspace_size(self.copies[0][0]),
+                   w4.i8_head_workspace_size(1, HEAD_K, HEAD_V))
         self.ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
         self.ws_bytes = self.ws.numel()
         self.lib = w4.lib()
@@ -199,9 +201,10 @@ class Workload:
             raise RuntimeError(f"w4_matmul_grouped failed: {st} {self.lib.w4_last_error()}")
 
     def head(self, r: int, stream_handle: int):
-        _, t, s = self.copies[r]
+        _, t, s, _ = self.copies[r]
         st = self.lib.i8_head_logits(self.h.data_ptr(), HEAD_K, t.data_ptr(), HEAD_V, s.data_ptr(),
-                                     self.logits.data_ptr(), HEAD_V, 1, HEAD_K, HEAD_V, stream_handle)
+                                     self.logits.data_ptr(), HEAD_V, 1, HEAD_K, HEAD_V, self.ws.data_ptr(),
+                                     self.ws_bytes, stream_handle)
         if st != 0:
             raise RuntimeError(f"i8_head_logits failed: {st} {self.lib.w4_last_error()}")
 

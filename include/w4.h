@@ -106,8 +106,9 @@ typedef struct w4_desc {
 /* ------------------------------------------------------------------ body */
 
 /* Bytes of workspace w4_matmul needs for this shape on the current device
- * (0 when none is needed). The workspace holds split-K partial sums and one
- * 32-bit counter per output tile. It must be device memory, 16-byte aligned,
+ * (0 when none is needed). The workspace starts with a fixed block of
+ * 32-bit split-K counters followed by partial sums. It must be device memory,
+ * 16-byte aligned,
  * and ZERO-FILLED before its first use; every successful call leaves it
  * zero-filled again, so one zeroing at allocation suffices. Two calls that
  * may run at the same time must not share a workspace. After a call that
@@ -140,18 +141,28 @@ W4_API w4_status w4_matmul_grouped(const w4_desc* descs, int32_t count, void* wo
 
 /* ------------------------------------------------------------------ head */
 
+/* Bytes of workspace i8_head_logits needs for this shape on the current
+ * device (same rules as w4_matmul's workspace: zero-filled before first use,
+ * left zero-filled by every successful call, not shared by calls that may run
+ * at the same time). One workspace of the larger size can serve both ops on
+ * one stream. */
+W4_API size_t i8_head_workspace_size(int64_t M, int64_t K, int64_t V);
+
 /* logits[M, V] = h[M, K] . (T[K, V] * s[V]); the M rows of h are the last
  * positions of M sequences (pass h = hidden + (T_len - 1) * ldh for one
  * sequence). Requires ldh >= K, ldt >= V, ldl >= V, h / scales / logits
- * 4-byte aligned, table 16-byte aligned. No workspace. */
+ * 4-byte aligned, table 16-byte aligned. workspace may be NULL only when
+ * i8_head_workspace_size() returns 0. */
 W4_API w4_status i8_head_logits(const float* h, int64_t ldh, const int8_t* table, int64_t ldt,
-                         const float* scales, float* logits, int64_t ldl, int64_t M, int64_t K,
-                         int64_t V, void* stream);
+                                const float* scales, float* logits, int64_t ldl, int64_t M, int64_t K,
+                                int64_t V, void* workspace, size_t workspace_bytes, void* stream);
 
-/* As i8_head_logits with an explicit kernel choice (AUTO, GEMV or GENERIC). */
+/* As i8_head_logits with an explicit kernel choice (AUTO, GEMV or GENERIC;
+ * the GENERIC kernel needs no workspace). */
 W4_API w4_status i8_head_logits_path(const float* h, int64_t ldh, const int8_t* table, int64_t ldt,
-                              const float* scales, float* logits, int64_t ldl, int64_t M,
-                              int64_t K, int64_t V, w4_path path, void* stream);
+                                     const float* scales, float* logits, int64_t ldl, int64_t M,
+                                     int64_t K, int64_t V, void* workspace, size_t workspace_bytes,
+                                     w4_path path, void* stream);
 
 /* ------------------------------------------------------------------ host packing */
 

@@ -87,9 +87,10 @@ def workspace(nbytes: int, device=None):
 
 
 def _ld(t, inner: int) -> int:
-    if t.dim() == 1:
-        return inner
-    if t.stride(-1) != 1:
+    """Row stride in elements; a single row has no stride of its own."""
+    if t.dim() == 1 or t.shape[0] <= 1:
+        return max(inner, 1)
+    if t.stride(-1) != 1 and t.shape[-1] > 1:
         raise ValueError("innermost dimension must be contiguous")
     return int(t.stride(0))
 
@@ -148,8 +149,12 @@ def w4_matmul_grouped(items: Sequence[dict] | None = None, descs=None, ws=None, 
 
 # ---------------------------------------------------------------- head
 
+def i8_head_workspace_size(M: int, K: int, V: int) -> int:
+    return int(lib().i8_head_workspace_size(M, K, V))
+
+
 def i8_head_logits(h, table, scales, K: int, V: int, ldt: int | None = None, logits=None, path: str = "auto",
-                   stream=None):
+                   ws=None, stream=None):
     """logits[M, V] = h[M, K] . (T[K, V] * s[V]) for the int8 tied head; h holds
     the last-position rows."""
     torch = _torch()
@@ -157,8 +162,12 @@ def i8_head_logits(h, table, scales, K: int, V: int, ldt: int | None = None, log
     ldt = V if ldt is None else ldt
     if logits is None:
         logits = torch.empty((M, V), dtype=torch.float32, device=h.device)
+    if ws is None:
+        ws = workspace(i8_head_workspace_size(M, K, V), h.device)
     st = lib().i8_head_logits_path(_ptr(h), _ld(h, K), _ptr(table), ldt, _ptr(scales), _ptr(logits),
-                                   _ld(logits, V), M, K, V, PATHS[path], _stream_handle(stream))
+                                   _ld(logits, V), M, K, V, _ptr(ws),
+                                   0 if ws is None else ws.numel() * ws.element_size(), PATHS[path],
+                                   _stream_handle(stream))
     _check(st, "i8_head_logits")
     return logits
 

@@ -7,11 +7,11 @@
 // Design (sm_100a):
 //  * Row k of T starts at byte k*ldt, which is not aligned when ldt is odd
 //    (V = 50257). With T 16-byte aligned, (k*ldt) mod 16 depends only on
-//    k mod 16, so a warp that takes the rows k = k0 + w + 16 i (w = warp)
-//    sees ONE misalignment r_w for all its rows. Each lane then loads
-//    aligned CB-byte chunks (LDG.128 for CB = 16) and the warp's 32 lanes
-//    cover the byte window that starts r_w bytes before the tile's first
-//    column: no realignment in registers at all. The CTA's reduction across
+//    k mod 16, so a warp that takes the rows k = 16 g + w (w = warp, g a
+//    16-row group) sees ONE misalignment r_w for all its rows. Each lane then
+//    loads aligned CB-byte chunks (LDG.128 for CB = 16) and the warp's 32
+//    lanes cover the byte window that starts r_w bytes before the tile's
+//    first column: no realignment in registers at all. The reduction across
 //    warps undoes the per-warp shift (column c of the tile sits at window
 //    position c + r_w of warp w). A tile is 31 chunks wide, so every warp's
 //    32-chunk window covers it whatever r_w is.
@@ -19,11 +19,12 @@
 //    0x80, is placed in the mantissa of 2^23 (0x4B0000uu), then one packed
 //    f32x2 add removes 2^23 + 128. The per-token scale is applied once per
 //    column after the sum.
-//  * K is split over a thread-block cluster of KS CTAs (grid.y); each CTA
-//    reduces its warps in shared memory, then CTA r of the cluster adds the
-//    KS partials of its share of the columns through distributed shared
-//    memory, in rank order (deterministic, no workspace, no atomics).
-#include <cooperative_groups.h>
+//  * Persistent stream-K, like the W4 GEMV: the units (16-row group of one
+//    column tile of one group of MT rows of h) form one flat range split
+//    evenly over the CTAs (one per SM). Each warp keeps the loads of the
+//    next D rows in flight while it converts and accumulates the current D. A tile whose rows straddle CTAs is finished by the last
+//    CTA to arrive, which adds the partials in CTA order (deterministic)
+//    through the caller's workspace and resets the counter to zero.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -31,23 +32,23 @@
 #include "w4_device.cuh"
 #include "w4_internal.h"
 
-namespace cg = cooperative_groups;
-
 namespace {
 
 using namespace w4dev;
 
-constexpr int NW = 16;  // warps per CTA; row stride of a warp
+constexpr int NW = 16;  // warps per CTA = rows per group (the alignment period)
+constexpr int COUNTER_SLOTS = 1024;
+constexpr size_t COUNTER_BYTES = COUNTER_SLOTS * sizeof(int32_t);
 
 template <int MT>
 struct HCfg {
   static constexpr int CB = MT <= 2 ? 16 : (MT == 4 ? 8 : 4);  // bytes per lane chunk
   static constexpr int WIN = 32 * CB;                          // window columns per warp
   static constexpr int TV = 31 * CB;                           // tile columns
-  static constexpr int D = MT == 8 ? 2 : 4;  // rows in flight per warp batch
+  static constexpr int D = MT == 1 ? 8 : (MT == 8 ? 2 : 4);   // rows per batch (two batches in flight)
+  static constexpr int MINB = 1;                               // CTAs per SM
   static constexpr int RED_FLOATS = NW * MT * WIN;
-  static constexpr int PART_FLOATS = MT * TV;
-  static constexpr int SMEM = (RED_FLOATS + PART_FLOATS) * 4 + 64 * 4;
+  static constexpr int SMEM = RED_FLOATS * 4 + NW * 4 + 16;
 };
 
 __device__ __forceinline__ float byte_magic(uint32_t biased_word, int j) {
@@ -78,7 +79,7 @@ __device__ __forceinline__ Chunk<CB> load_chunk(const int8_t* p) {
 // Bytes of a chunk that straddles the end of the table: read the ones before
 // `end`, zero the rest (their columns are never written).
 template <int CB>
-__device__ __forceinline__ Chunk<CB> load_chunk_clipped(const int8_t* p, const int8_t* end) {
+__device__ __noinline__ Chunk<CB> load_chunk_clipped(const int8_t* p, const int8_t* end) {
   Chunk<CB> c;
 #pragma unroll
   for (int i = 0; i < CB / 4; ++i) {
@@ -94,118 +95,217 @@ __device__ __forceinline__ Chunk<CB> load_chunk_clipped(const int8_t* p, const i
   return c;
 }
 
+struct HeadParams {
+  const float* h;
+  int64_t ldh;
+  const int8_t* table;
+  int64_t ldt;
+  const float* scales;
+  float* logits;
+  int64_t ldl;
+  int32_t M, K, V;
+  int32_t ntiles, NG, nmc;
+  int64_t U;  // total units
+  int32_t* ws_counters;
+  float* ws_partials;  // [grid][2][MT][TV]
+};
+
+__device__ __forceinline__ int64_t cta_of(int64_t f, int64_t W, int64_t G) { return ((f + 1) * G + W - 1) / W - 1; }
+__device__ __forceinline__ int64_t range_lo(int64_t i, int64_t W, int64_t G) { return (i * W) / G; }
+
 template <int MT>
-__global__ void __launch_bounds__(NW * 32, MT == 1 ? 2 : 1) i8_head_kernel(const float* __restrict__ h, int64_t ldh,
-                                                             const int8_t* __restrict__ table, int64_t ldt,
-                                                             const float* __restrict__ scales,
-                                                             float* __restrict__ logits, int64_t ldl, int32_t M,
-                                                             int32_t K, int32_t V, int32_t KR) {
+__global__ void __launch_bounds__(NW * 32, HCfg<MT>::MINB) i8_head_kernel(const __grid_constant__ HeadParams p) {
   using C = HCfg<MT>;
   constexpr int CB = C::CB;
   extern __shared__ __align__(16) float hsm[];
-  float* red = hsm;                       // [NW][MT][WIN]
-  float* part = hsm + C::RED_FLOATS;      // [MT][TV]
-  int* shift = reinterpret_cast<int*>(part + C::PART_FLOATS);  // [NW]
+  float* red = hsm;                                          // [NW][MT][WIN]
+  int* shift = reinterpret_cast<int*>(hsm + C::RED_FLOATS);  // [NW]
+  int* bcast = shift + NW;
 
-  cg::cluster_group cluster = cg::this_cluster();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * C::TV;
-  const int32_t kbeg = blockIdx.y * KR;
-  const int32_t kend = min(K, kbeg + KR);
-  const int32_t m0 = blockIdx.z * MT;
-  const int mrows = min(MT, M - m0);
-  const int8_t* table_end = table + (static_cast<int64_t>(K) - 1) * ldt + V;
-
-  // window of this warp: starts r bytes before column v0 of each of its rows
-  const int64_t first_row = kbeg + warp;
-  const int r = static_cast<int>(reinterpret_cast<uintptr_t>(table + first_row * ldt + v0) & (CB - 1));
-  if (lane == 0) shift[warp] = r;
-
-  // acc[mm * CB/2 + pp] = columns {2pp, 2pp+1} of the lane's chunk, row mm
-  float2 acc[MT * CB / 2];
-#pragma unroll
-  for (int i = 0; i < MT * CB / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+  const int64_t G = gridDim.x;
+  const int64_t lo = range_lo(blockIdx.x, p.U, G);
+  const int64_t hi = range_lo(blockIdx.x + 1, p.U, G);
+  const int8_t* table_end = p.table + (static_cast<int64_t>(p.K) - 1) * p.ldt + p.V;
   const float2 bias = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
 
-  for (int32_t k0 = kbeg + warp; k0 < kend; k0 += NW * C::D) {
-    Chunk<CB> ch[C::D];
-    float hv[C::D][MT];
+  int64_t f = lo;
+  while (f < hi) {
+    const int64_t tile_l = f / p.NG;  // = mc * ntiles + tile
+    const int32_t g0 = static_cast<int32_t>(f - tile_l * p.NG);
+    const int64_t seg_end = min(hi, (tile_l + 1) * p.NG);
+    const int32_t g1 = static_cast<int32_t>(seg_end - tile_l * p.NG);
+    const int32_t mc = static_cast<int32_t>(tile_l / p.ntiles);
+    const int32_t tile = static_cast<int32_t>(tile_l - static_cast<int64_t>(mc) * p.ntiles);
+    const int64_t v0 = static_cast<int64_t>(tile) * C::TV;
+    const int32_t m0 = mc * MT;
+    const int mrows = min(MT, p.M - m0);
+
+    // this warp's rows: k = 16 g + warp, g in [g0, g1), k < K; one window shift
+    const int r = static_cast<int>(
+        reinterpret_cast<uintptr_t>(p.table + (static_cast<int64_t>(g0) * NW + warp) * p.ldt + v0) & (CB - 1));
+    const int8_t* wbase = p.table + v0 - r + lane * CB;
+
+    float2 acc[MT * CB / 2];
 #pragma unroll
-    for (int j = 0; j < C::D; ++j) {
-      const int32_t k = k0 + j * NW;
-      if (k < kend) {
-        const int8_t* p = table + static_cast<int64_t>(k) * ldt + v0 - r + lane * CB;
-        ch[j] = (p + CB <= table_end) ? load_chunk<CB>(p) : load_chunk_clipped<CB>(p, table_end);
+    for (int i = 0; i < MT * CB / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+
+    // Software pipeline: the loads of the next D rows are in flight while the
+    // current D rows are converted and accumulated.
+    // Whether a batch's windows can reach past the end of the table is decided
+    // once per batch for the whole warp (the window of row k ends at
+    // win_end0 + k * ldt), so the usual path carries no per-row bounds logic.
+    const int8_t* win_end0 = p.table + v0 - r + 32 * CB;
+    auto load_batch = [&](int32_t gb, Chunk<CB> (&ch)[C::D], float (&hv)[C::D][MT]) {
+      const int64_t k_hi = min(static_cast<int64_t>(gb + C::D) * NW - 1, static_cast<int64_t>(p.K) - 1);
+      const bool careful = win_end0 + k_hi * p.ldt > table_end;
+      if (!careful) {
+        const bool full = (gb + C::D <= g1) && ((gb + C::D) * NW <= p.K);
+        if (full) {
 #pragma unroll
-        for (int mm = 0; mm < MT; ++mm)
-          hv[j][mm] = (mm < mrows) ? __ldg(h + static_cast<int64_t>(m0 + mm) * ldh + k) : 0.f;
-      } else {
+          for (int j = 0; j < C::D; ++j) {
+            const int32_t k = (gb + j) * NW + warp;
+            ch[j] = load_chunk<CB>(wbase + static_cast<int64_t>(k) * p.ldt);
 #pragma unroll
-        for (int i = 0; i < CB / 4; ++i) ch[j].w[i] = 0u;  // q = 0
-#pragma unroll
-        for (int mm = 0; mm < MT; ++mm) hv[j][mm] = 0.f;
+            for (int mm = 0; mm < MT; ++mm)
+              hv[j][mm] = (mm < mrows) ? __ldg(p.h + static_cast<int64_t>(m0 + mm) * p.ldh + k) : 0.f;
+          }
+          return;
+        }
       }
-    }
 #pragma unroll
-    for (int j = 0; j < C::D; ++j) {
+      for (int j = 0; j < C::D; ++j) {
+        const int32_t k = (gb + j) * NW + warp;
+        if (gb + j < g1 && k < p.K) {
+          const int8_t* q = wbase + static_cast<int64_t>(k) * p.ldt;
+          ch[j] = (!careful || q + CB <= table_end) ? load_chunk<CB>(q) : load_chunk_clipped<CB>(q, table_end);
 #pragma unroll
-      for (int i = 0; i < CB / 4; ++i) {
-        const uint32_t bw = ch[j].w[i] ^ 0x80808080u;
+          for (int mm = 0; mm < MT; ++mm)
+            hv[j][mm] = (mm < mrows) ? __ldg(p.h + static_cast<int64_t>(m0 + mm) * p.ldh + k) : 0.f;
+        } else {
 #pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
-          const float2 e = make_float2(byte_magic(bw, 2 * pr), byte_magic(bw, 2 * pr + 1));
-          const float2 q = __fadd2_rn(e, bias);  // exact int8 values
+          for (int i = 0; i < CB / 4; ++i) ch[j].w[i] = 0u;  // q = 0
 #pragma unroll
-          for (int mm = 0; mm < MT; ++mm) {
-            const float2 hh = make_float2(hv[j][mm], hv[j][mm]);
-            acc[mm * (CB / 2) + i * 2 + pr] = __ffma2_rn(hh, q, acc[mm * (CB / 2) + i * 2 + pr]);
+          for (int mm = 0; mm < MT; ++mm) hv[j][mm] = 0.f;
+        }
+      }
+    };
+    Chunk<CB> cur[C::D];
+    float hcur[C::D][MT];
+    load_batch(g0, cur, hcur);
+    for (int32_t gb = g0; gb < g1; gb += C::D) {
+      Chunk<CB> nxt[C::D];
+      float hnxt[C::D][MT];
+      if (gb + C::D < g1) load_batch(gb + C::D, nxt, hnxt);
+#pragma unroll
+      for (int j = 0; j < C::D; ++j) {
+#pragma unroll
+        for (int i = 0; i < CB / 4; ++i) {
+          const uint32_t bw = cur[j].w[i] ^ 0x80808080u;
+#pragma unroll
+          for (int pr = 0; pr < 2; ++pr) {
+            const float2 e = make_float2(byte_magic(bw, 2 * pr), byte_magic(bw, 2 * pr + 1));
+            const float2 qv = __fadd2_rn(e, bias);  // exact int8 values
+#pragma unroll
+            for (int mm = 0; mm < MT; ++mm) {
+              const float2 hh = make_float2(hcur[j][mm], hcur[j][mm]);
+              acc[mm * (CB / 2) + i * 2 + pr] = __ffma2_rn(hh, qv, acc[mm * (CB / 2) + i * 2 + pr]);
+            }
           }
         }
       }
+      if (gb + C::D < g1) {
+#pragma unroll
+        for (int j = 0; j < C::D; ++j) {
+          cur[j] = nxt[j];
+#pragma unroll
+          for (int mm = 0; mm < MT; ++mm) hcur[j][mm] = hnxt[j][mm];
+        }
+      }
     }
-  }
 
-  // ---- CTA reduction across warps (undo the per-warp window shift)
+    // ---- reduce the warps (undoing each warp's window shift)
 #pragma unroll
-  for (int mm = 0; mm < MT; ++mm) {
-    float* dst = red + (warp * MT + mm) * C::WIN + lane * CB;
+    for (int mm = 0; mm < MT; ++mm) {
+      float* dst = red + (warp * MT + mm) * C::WIN + lane * CB;
 #pragma unroll
-    for (int pp = 0; pp < CB / 2; ++pp) {
-      dst[2 * pp] = acc[mm * (CB / 2) + pp].x;
-      dst[2 * pp + 1] = acc[mm * (CB / 2) + pp].y;
+      for (int pp = 0; pp < CB / 2; ++pp) {
+        dst[2 * pp] = acc[mm * (CB / 2) + pp].x;
+        dst[2 * pp + 1] = acc[mm * (CB / 2) + pp].y;
+      }
     }
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < MT * C::TV; idx += NW * 32) {
-    const int mm = idx / C::TV;
-    const int c = idx - mm * C::TV;
-    float v = 0.f;
+    if (lane == 0) shift[warp] = r;
+    __syncthreads();
+
+    const int64_t t_start = tile_l * p.NG;
+    const int64_t c_first = cta_of(t_start, p.U, G);
+    const int64_t c_last = cta_of(t_start + p.NG - 1, p.U, G);
+    const bool split = c_first != c_last;
+    const int slot = (split && static_cast<int64_t>(blockIdx.x) == c_first && lo < t_start) ? 1 : 0;
+    for (int idx = threadIdx.x; idx < MT * C::TV; idx += NW * 32) {
+      const int mm = idx / C::TV;
+      const int c = idx - mm * C::TV;
+      float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) v += red[(w * MT + mm) * C::WIN + c + shift[w]];
-    part[idx] = v;
+      for (int w = 0; w < NW; ++w) v += red[(w * MT + mm) * C::WIN + c + shift[w]];
+      const int64_t col = v0 + c;
+      if (!split) {
+        if (mm < mrows && col < p.V) p.logits[static_cast<int64_t>(m0 + mm) * p.ldl + col] = v * __ldg(p.scales + col);
+      } else {
+        p.ws_partials[((static_cast<int64_t>(blockIdx.x) * 2 + slot) * MT + mm) * C::TV + c] = v;
+      }
+    }
+    if (split) {
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) bcast[0] = atomicAdd(&p.ws_counters[c_first], 1);
+      __syncthreads();
+      if (bcast[0] == static_cast<int>(c_last - c_first)) {
+        __threadfence();
+        for (int idx = threadIdx.x; idx < MT * C::TV; idx += NW * 32) {
+          const int mm = idx / C::TV;
+          const int c = idx - mm * C::TV;
+          float v = 0.f;
+          for (int64_t cc = c_first; cc <= c_last; ++cc) {
+            const int sl = (cc == c_first && range_lo(cc, p.U, G) < t_start) ? 1 : 0;
+            v += __ldcg(&p.ws_partials[((cc * 2 + sl) * MT + mm) * C::TV + c]);
+          }
+          const int64_t col = v0 + c;
+          if (mm < mrows && col < p.V)
+            p.logits[static_cast<int64_t>(m0 + mm) * p.ldl + col] = v * __ldg(p.scales + col);
+        }
+        if (threadIdx.x == 0) p.ws_counters[c_first] = 0;
+      }
+    }
+    __syncthreads();  // red / shift are reused by the next segment
+    f = seg_end;
   }
-  // ---- cluster reduction across the K-split, through distributed shared memory
-  cluster.sync();
-  const int ks = static_cast<int>(cluster.num_blocks());
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int per = (C::TV + ks - 1) / ks;
-  const int c_lo = rank * per;
-  const int c_hi = min(C::TV, c_lo + per);
-  for (int idx = threadIdx.x; idx < MT * per; idx += NW * 32) {
-    const int mm = idx / per;
-    const int c = c_lo + (idx - mm * per);
-    if (c >= c_hi) continue;
-    float v = 0.f;
-    for (int q = 0; q < ks; ++q) v += cluster.map_shared_rank(part, q)[mm * C::TV + c];
-    const int64_t col = v0 + c;
-    if (mm < mrows && col < V) logits[static_cast<int64_t>(m0 + mm) * ldl + col] = v * __ldg(scales + col);
-  }
-  cluster.sync();  // keep this CTA's shared memory alive until every peer has read it
+}
+
+struct HPlan {
+  int mt;
+  int tv;
+  int64_t ntiles, NG, nmc, U;
+  int grid;
+};
+
+HPlan head_plan(int64_t M, int64_t K, int64_t V, int sms) {
+  HPlan pl;
+  pl.mt = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
+  const int cb = pl.mt <= 2 ? 16 : (pl.mt == 4 ? 8 : 4);
+  pl.tv = 31 * cb;
+  pl.ntiles = (V + pl.tv - 1) / pl.tv;
+  pl.NG = (K + NW - 1) / NW;
+  pl.nmc = (M + pl.mt - 1) / pl.mt;
+  pl.U = pl.ntiles * pl.NG * pl.nmc;
+  const int per_sm = 1;
+  pl.grid = static_cast<int>(std::min<int64_t>(std::min(per_sm * sms, COUNTER_SLOTS), pl.U));
+  return pl;
 }
 
 template <int MT>
-w4_status launch_head_mt(const w4host::HeadArgs& a, cudaStream_t st, const w4host::DeviceInfo& di) {
+w4_status launch_head_mt(const HeadParams& prm, int grid, cudaStream_t st, const w4host::DeviceInfo& di) {
   using C = HCfg<MT>;
   static int configured[64] = {};
   if (di.dev < 64 && !configured[di.dev]) {
@@ -213,46 +313,53 @@ w4_status launch_head_mt(const w4host::HeadArgs& a, cudaStream_t st, const w4hos
     if (e != cudaSuccess) return w4host::cuda_fail(e, "cudaFuncSetAttribute(i8_head)");
     configured[di.dev] = 1;
   }
-  const int64_t ntiles = (a.V + C::TV - 1) / C::TV;
-  const int64_t nmc = (a.M + MT - 1) / MT;
-  // K-split: enough CTAs for two per SM, at most 8 (portable cluster size),
-  // at least 16 rows (one per warp) per CTA.
-  int ks = static_cast<int>((2 * di.sms + ntiles * nmc - 1) / (ntiles * nmc));
-  ks = std::max(1, std::min({ks, 8, static_cast<int>((a.K + NW - 1) / NW)}));
-  const int32_t KR = static_cast<int32_t>(((a.K + ks - 1) / ks + NW - 1) / NW * NW);
-  ks = static_cast<int>((a.K + KR - 1) / KR);
-  if (ntiles > 0x7fffffff || nmc > 65535) return w4host::fail(W4_ERR_SHAPE, "head grid too large");
-
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(ntiles), static_cast<unsigned>(ks), static_cast<unsigned>(nmc));
-  cfg.blockDim = dim3(NW * 32, 1, 1);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = static_cast<unsigned>(ks);
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, i8_head_kernel<MT>, a.h, a.ldh, a.table, a.ldt, a.scales, a.logits, a.ldl,
-                                     static_cast<int32_t>(a.M), static_cast<int32_t>(a.K), static_cast<int32_t>(a.V),
-                                     KR);
-  if (e != cudaSuccess) return w4host::cuda_fail(e, "launch i8_head");
-  return W4_OK;
+  i8_head_kernel<MT><<<grid, NW * 32, C::SMEM, st>>>(prm);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W4_OK : w4host::cuda_fail(e, "launch i8_head");
 }
 
 }  // namespace
 
 namespace w4host {
 
-w4_status launch_head(const HeadArgs& a, cudaStream_t st, const DeviceInfo& di) {
+size_t head_workspace_bytes(int64_t M, int64_t K, int64_t V, int sms) {
+  if (M <= 0 || K <= 0 || V <= 0) return 0;
+  const HPlan pl = head_plan(M, K, V, sms);
+  return COUNTER_BYTES + static_cast<size_t>(pl.grid) * 2 * pl.mt * pl.tv * sizeof(float);
+}
+
+w4_status launch_head(const HeadArgs& a, void* ws, size_t ws_size, cudaStream_t st, const DeviceInfo& di) {
   if (a.K > 0x7fffffff || a.V > 0x7fffffff || a.M > 0x7fffffff)
     return fail(W4_ERR_SHAPE, "head sizes must be below 2^31 on the fast path");
-  if (a.M <= 1) return launch_head_mt<1>(a, st, di);
-  if (a.M <= 2) return launch_head_mt<2>(a, st, di);
-  if (a.M <= 4) return launch_head_mt<4>(a, st, di);
-  return launch_head_mt<8>(a, st, di);
+  const HPlan pl = head_plan(a.M, a.K, a.V, di.sms);
+  const size_t need = head_workspace_bytes(a.M, a.K, a.V, di.sms);
+  if (ws == nullptr || ws_size < need)
+    return fail(W4_ERR_WORKSPACE, "head workspace of %zu bytes needed, %zu given", need,
+                ws == nullptr ? size_t(0) : ws_size);
+  if ((reinterpret_cast<uintptr_t>(ws) & 15) != 0) return fail(W4_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+  HeadParams prm;
+  prm.h = a.h;
+  prm.ldh = a.ldh;
+  prm.table = a.table;
+  prm.ldt = a.ldt;
+  prm.scales = a.scales;
+  prm.logits = a.logits;
+  prm.ldl = a.ldl;
+  prm.M = static_cast<int32_t>(a.M);
+  prm.K = static_cast<int32_t>(a.K);
+  prm.V = static_cast<int32_t>(a.V);
+  prm.ntiles = static_cast<int32_t>(pl.ntiles);
+  prm.NG = static_cast<int32_t>(pl.NG);
+  prm.nmc = static_cast<int32_t>(pl.nmc);
+  prm.U = pl.U;
+  prm.ws_counters = static_cast<int32_t*>(ws);
+  prm.ws_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + COUNTER_BYTES);
+  switch (pl.mt) {
+    case 1: return launch_head_mt<1>(prm, pl.grid, st, di);
+    case 2: return launch_head_mt<2>(prm, pl.grid, st, di);
+    case 4: return launch_head_mt<4>(prm, pl.grid, st, di);
+    default: return launch_head_mt<8>(prm, pl.grid, st, di);
+  }
 }
 
 }  // namespace w4host

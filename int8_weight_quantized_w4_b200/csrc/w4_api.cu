@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
+#include <unordered_map>
 
 #include "w4_device.cuh"
 #include "w4_internal.h"
@@ -92,7 +93,66 @@ w4_status current_device(const DeviceInfo** out) {
   return W4_OK;
 }
 
-w4_status encode_qw_map(CUtensorMap* map, const uint8_t* qw, int64_t K, int64_t N) {
+static w4_status encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                           uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(W4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): dims %llu x %llu, box %u x %u", int(r),
+                (unsigned long long)inner, (unsigned long long)rows, box_inner, box_rows);
+  return W4_OK;
+}
+
+namespace {
+struct MapKey {
+  const void* qw;
+  const void* sc;
+  const void* zp;
+  int64_t K, N;
+  bool operator==(const MapKey& o) const {
+    return qw == o.qw && sc == o.sc && zp == o.zp && K == o.K && N == o.N;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    size_t h = reinterpret_cast<size_t>(k.qw) * 0x9E3779B97F4A7C15ull;
+    h ^= reinterpret_cast<size_t>(k.sc) + 0x7F4A7C159E3779B9ull + (h << 6) + (h >> 2);
+    h ^= reinterpret_cast<size_t>(k.zp) + (h << 6) + (h >> 2);
+    h ^= static_cast<size_t>(k.K) * 31 + static_cast<size_t>(k.N) + (h << 6) + (h >> 2);
+    return h;
+  }
+};
+struct MapSet {
+  CUtensorMap m[4];
+};
+std::mutex g_map_mu;
+std::unordered_map<MapKey, MapSet, MapKeyHash> g_map_cache;
+constexpr size_t kMapCacheMax = 4096;
+}  // namespace
+
+// The four tensor maps of one packed weight (the GEMV's copies). A map is a
+// pure function of (pointers, K, N), so the cache can never return a stale
+// one: reusing freed memory for another weight of the same shape yields the
+// same map.
+w4_status encode_w4_maps(CUtensorMap* qw_full, CUtensorMap* qw_blk, CUtensorMap* sc_full, CUtensorMap* zp_full,
+                         const uint8_t* qw, const float* scales, const uint8_t* zp, int64_t K, int64_t N) {
+  const MapKey key{qw, scales, zp, K, N};
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    auto itc = g_map_cache.find(key);
+    if (itc != g_map_cache.end()) {
+      *qw_full = itc->second.m[0];
+      *qw_blk = itc->second.m[1];
+      *sc_full = itc->second.m[2];
+      *zp_full = itc->second.m[3];
+      return W4_OK;
+    }
+  }
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -102,15 +162,20 @@ w4_status encode_qw_map(CUtensorMap* map, const uint8_t* qw, int64_t K, int64_t 
       g_encode = reinterpret_cast<EncodeTiledFn>(fn);
   });
   if (g_encode == nullptr) return fail(W4_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N / 2), static_cast<cuuint64_t>(K)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N / 2)};
-  const cuuint32_t box[2] = {128, 32};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(qw), dims, strides, box,
-                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for K=%lld N=%lld", int(r),
-                                     (long long)K, (long long)N);
+  const uint64_t half = static_cast<uint64_t>(N / 2), nb = static_cast<uint64_t>(K / 32);
+  MapSet ms;
+  w4_status rc;
+  if ((rc = encode_2d(&ms.m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, half, K, half, 128, 256)) != W4_OK) return rc;
+  if ((rc = encode_2d(&ms.m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, half, K, half, 128, 32)) != W4_OK) return rc;
+  if ((rc = encode_2d(&ms.m[2], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, scales, N, nb, N * 4, 256, 8)) != W4_OK) return rc;
+  if ((rc = encode_2d(&ms.m[3], CU_TENSOR_MAP_DATA_TYPE_UINT8, zp, half, nb, half, 128, 8)) != W4_OK) return rc;
+  *qw_full = ms.m[0];
+  *qw_blk = ms.m[1];
+  *sc_full = ms.m[2];
+  *zp_full = ms.m[3];
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  if (g_map_cache.size() >= kMapCacheMax) g_map_cache.clear();
+  g_map_cache.emplace(key, ms);
   return W4_OK;
 }
 
@@ -290,7 +355,7 @@ w4_status w4_matmul_grouped(const w4_desc* descs, int32_t count, void* workspace
 
 // ------------------------------------------------------------------ head
 
-static w4_status head_impl(const HeadArgs& a, w4_path path, cudaStream_t st) {
+static w4_status head_impl(const HeadArgs& a, void* ws, size_t wsb, w4_path path, cudaStream_t st) {
   if (a.M < 0 || a.K < 0 || a.V < 0) return fail(W4_ERR_SHAPE, "negative size");
   if (path != W4_PATH_AUTO && path != W4_PATH_GEMV && path != W4_PATH_GENERIC)
     return fail(W4_ERR_VALUE, "path %d is not a head path", int(path));
@@ -311,19 +376,27 @@ static w4_status head_impl(const HeadArgs& a, w4_path path, cudaStream_t st) {
   if (rc != W4_OK) return rc;
   if (a.K == 0) return launch_zero_fill(a.logits, a.ldl, a.M, a.V, st);
   if (path == W4_PATH_GENERIC) return launch_head_generic(a, st, *di);
-  return launch_head(a, st, *di);
+  return launch_head(a, ws, wsb, st, *di);
+}
+
+size_t i8_head_workspace_size(int64_t M, int64_t K, int64_t V) {
+  const DeviceInfo* di = nullptr;
+  if (current_device(&di) != W4_OK) return 0;
+  return head_workspace_bytes(M, K, V, di->sms);
 }
 
 w4_status i8_head_logits_path(const float* h, int64_t ldh, const int8_t* table, int64_t ldt, const float* scales,
-                              float* logits, int64_t ldl, int64_t M, int64_t K, int64_t V, w4_path path,
-                              void* stream) {
+                              float* logits, int64_t ldl, int64_t M, int64_t K, int64_t V, void* workspace,
+                              size_t workspace_bytes, w4_path path, void* stream) {
   const HeadArgs a = {h, ldh, table, ldt, scales, logits, ldl, M, K, V};
-  return head_impl(a, path, static_cast<cudaStream_t>(stream));
+  return head_impl(a, workspace, workspace_bytes, path, static_cast<cudaStream_t>(stream));
 }
 
 w4_status i8_head_logits(const float* h, int64_t ldh, const int8_t* table, int64_t ldt, const float* scales,
-                         float* logits, int64_t ldl, int64_t M, int64_t K, int64_t V, void* stream) {
-  return i8_head_logits_path(h, ldh, table, ldt, scales, logits, ldl, M, K, V, W4_PATH_AUTO, stream);
+                         float* logits, int64_t ldl, int64_t M, int64_t K, int64_t V, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return i8_head_logits_path(h, ldh, table, ldt, scales, logits, ldl, M, K, V, workspace, workspace_bytes,
+                             W4_PATH_AUTO, stream);
 }
 
 // ------------------------------------------------------------------ diagnostics

@@ -76,24 +76,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with parity `parity` of `bar` has completed. Returns
-// false (after recording the error) when `timeout_ns` passes first, or at
-// once when *abort is already set by another thread of the CTA.
+// false (after recording the error) when `timeout_ns` passes first, or when
+// *abort is set by another thread of the CTA. The timer and the abort flag
+// are looked at once every 1024 polls, so a waiting warp costs few issue
+// slots (try_wait itself suspends the thread for a while when the phase is
+// not complete).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
                                                   volatile int* abort, ErrorWord* err, int32_t kernel,
                                                   int32_t detail) {
   const uint32_t a = smem_u32(bar);
-#pragma unroll 1
-  for (int i = 0; i < 32; ++i)
-    if (mbar_try_wait(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  if (mbar_try_wait(a, parity)) return true;
+  uint64_t t0 = 0;
+  uint32_t n = 0;
 #pragma unroll 1
   while (true) {
     if (mbar_try_wait(a, parity)) return true;
-    if (abort != nullptr && *abort) return false;
-    if (globaltimer_ns() - t0 > timeout_ns) {
-      if (abort != nullptr) *abort = 1;
-      record_error(err, W4_ERR_TIMEOUT, kernel, detail);
-      return false;
+    if ((++n & 1023u) == 0) {
+      if (abort != nullptr && *abort) return false;
+      const uint64_t t = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = t;
+      } else if (t - t0 > timeout_ns) {
+        if (abort != nullptr) *abort = 1;
+        record_error(err, W4_ERR_TIMEOUT, kernel, detail);
+        return false;
+      }
     }
   }
 }

@@ -12,12 +12,18 @@
 //    CTA to arrive: each writes its partial sums to the workspace, bumps the
 //    tile's counter, and the last one adds the partials in CTA order (a fixed
 //    order: the result does not depend on arrival order) and resets the
-//    counter to zero.
-//  * Warp-specialised: warp 0 is the producer. One lane issues, per K-block,
-//    a 2-D tensor copy of the nibbles (32 rows x 128 B), and untiled bulk
-//    copies of the block's scales, zero points and x values into a ring of
-//    shared-memory stages guarded by mbarriers (no multicast). The consumer
-//    warps dequantise in registers and accumulate.
+//    counter to zero. A CTA is the first contributor of at most one split
+//    tile, so counters are indexed by that CTA and live in a fixed region at
+//    the start of the workspace: whatever shapes earlier calls had, the
+//    counter region is all zeros between calls.
+//  * Warp-specialised: warp 0 is the producer. Stages hold 8 K-blocks and
+//    are aligned to the tile's 8-block grid, so a full stage is four copies,
+//    issued by four lanes at once: 2-D tensor copies of the nibbles
+//    (256 rows x 128 B), the scales (8 x 256 fp32) and the zero points
+//    (8 x 128 B), and an untiled bulk copy per row of x. A partial stage (at
+//    the ends of a CTA's range) issues per-block copies, one lane per block.
+//    The stages form a ring guarded by mbarriers (no multicast anywhere).
+//    The consumer warps dequantise in registers and accumulate.
 //  * Dequantisation uses the exponent trick of w4_device.cuh: one LOP3 per
 //    weight builds 2^23 + q*16^j, one packed f32x2 add subtracts the matching
 //    zero-point float, packed f32x2 FMAs accumulate. Lane l owns 8 columns
@@ -46,8 +52,10 @@ constexpr int QW_STAGE = SB * 32 * (TILE_N / 2);  // 32 KB
 constexpr int SC_STAGE = SB * TILE_N * 4;         // 8 KB
 constexpr int ZP_STAGE = SB * (TILE_N / 2);       // 1 KB
 
-struct MatParams {
-  CUtensorMap qw_map;  // [K rows][N/2 bytes], box 32 rows x 128 bytes
+// Per-matrix fields the kernel reads while walking its range. They are copied
+// from the parameter block into shared memory once per CTA: dynamically
+// indexed reads of a large parameter block miss the constant cache.
+struct MatScalars {
   const float* x;
   const float* scales;
   const uint8_t* zp;
@@ -56,10 +64,17 @@ struct MatParams {
   int64_t ldy;
   int64_t bt_off;  // first flat block-tile of this matrix
   int32_t M, K, N, nb;
-  int32_t ntn;       // column tiles
-  int32_t nmc;       // groups of MT rows
-  int32_t tile_off;  // first global tile index
-  int32_t pad;
+  int32_t ntn;  // column tiles
+  int32_t nmc;  // groups of MT rows
+};
+static_assert(sizeof(MatScalars) % 8 == 0, "copied as 8-byte words");
+
+struct MatParams {
+  CUtensorMap qw_full;  // [K rows][N/2 bytes], box 256 rows x 128 bytes
+  CUtensorMap qw_blk;   // same tensor, box 32 rows x 128 bytes
+  CUtensorMap sc_full;  // [K/32][N] fp32, box 8 x 256
+  CUtensorMap zp_full;  // [K/32][N/2 bytes], box 8 x 128
+  MatScalars s;
 };
 
 struct GemvParams {
@@ -85,7 +100,8 @@ struct Cfg {
   // per-warp column sums: [NCW][TILE_N] reused per row (register accumulator)
   // or [NCW][MT][TILE_N] holding the accumulator itself (SMEM_ACC)
   static constexpr int RED_BYTES = NCW * (SMEM_ACC ? MT : 1) * TILE_N * 4;
-  static constexpr int BAR_OFF = NSTAGES * STAGE_BYTES + RED_BYTES;
+  static constexpr int SCAL_OFF = NSTAGES * STAGE_BYTES + RED_BYTES;
+  static constexpr int BAR_OFF = SCAL_OFF + W4_GROUP_MAX * static_cast<int>(sizeof(MatScalars));
   static constexpr int SMEM_BYTES = BAR_OFF + 2 * NSTAGES * 8 + 64;
 };
 
@@ -96,11 +112,11 @@ struct Pos {
   int32_t blk;
 };
 
-__device__ __forceinline__ Pos locate(const GemvParams& p, int64_t f) {
-  int g = 0;
+__device__ __forceinline__ Pos locate(const MatScalars* ms, int count, int64_t f, int g_hint) {
+  int g = g_hint;
 #pragma unroll 1
-  while (g + 1 < p.count && p.mat[g + 1].bt_off <= f) ++g;
-  const MatParams& m = p.mat[g];
+  while (g + 1 < count && ms[g + 1].bt_off <= f) ++g;
+  const MatScalars& m = ms[g];
   const int64_t local = f - m.bt_off;
   Pos r;
   r.g = g;
@@ -123,6 +139,7 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::NSTAGES);
   int* bcast = reinterpret_cast<int*>(empty + C::NSTAGES) + 4;
   float* red = reinterpret_cast<float*>(smem + C::NSTAGES * C::STAGE_BYTES);
+  MatScalars* ms = reinterpret_cast<MatScalars*>(smem + C::SCAL_OFF);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -138,62 +155,91 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
     *abort_flag = 0;
     fence_mbar_init();
   }
+  {
+    constexpr int WORDS = sizeof(MatScalars) / 8;
+    for (int i = threadIdx.x; i < p.count * WORDS; i += blockDim.x) {
+      const int g = i / WORDS, j = i - g * WORDS;
+      reinterpret_cast<uint64_t*>(ms + g)[j] = reinterpret_cast<const uint64_t*>(&p.mat[g].s)[j];
+    }
+  }
   __syncthreads();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane != 0) return;
-    for (int g = 0; g < p.count; ++g) prefetch_tensormap(&p.mat[g].qw_map);
+    if (lo < hi) {
+      const int g_first = locate(ms, p.count, lo, 0).g;
+      const int g_last = locate(ms, p.count, hi - 1, g_first).g;
+      for (int g = g_first + (lane >> 2); g <= g_last; g += 8) {
+        const CUtensorMap* mp = (lane & 3) == 0 ? &p.mat[g].qw_full
+                               : (lane & 3) == 1 ? &p.mat[g].qw_blk
+                               : (lane & 3) == 2 ? &p.mat[g].sc_full : &p.mat[g].zp_full;
+        prefetch_tensormap(mp);
+      }
+    }
     int it = 0;
+    int g_hint = 0;
     bool ok = true;
     int64_t f = lo;
     while (f < hi && ok) {
-      const Pos ps = locate(p, f);
-      const MatParams& m = p.mat[ps.g];
+      const Pos ps = locate(ms, p.count, f, g_hint);
+      g_hint = ps.g;
+      const MatScalars& m = ms[ps.g];
+      const MatParams& mp = p.mat[ps.g];
       const int64_t seg_end = min(hi, f + (m.nb - ps.blk));
       const int32_t t = static_cast<int32_t>(ps.tile_l / m.nmc);
       const int32_t mc = static_cast<int32_t>(ps.tile_l - static_cast<int64_t>(t) * m.nmc);
       const int32_t ncols = min(TILE_N, m.N - t * TILE_N);
       const int32_t mrows = min(MT, m.M - mc * MT);
+      const float* xrow0 = m.x + static_cast<int64_t>(mc) * MT * m.ldx;
+      const float* scol = m.scales + static_cast<int64_t>(t) * TILE_N;
+      const uint8_t* zcol = m.zp + static_cast<int64_t>(t) * (TILE_N / 2);
       int32_t blk = ps.blk;
-      for (int64_t cur = f; cur < seg_end; ) {
-        const int32_t nblk = static_cast<int32_t>(min(static_cast<int64_t>(SB), seg_end - cur));
+      const int32_t blk_end = blk + static_cast<int32_t>(seg_end - f);
+      while (blk < blk_end) {
+        const int32_t nblk = min(SB - (blk % SB), blk_end - blk);  // stay on the 8-block grid
+        const bool full_stage = (nblk == SB);
         const int s = it % C::NSTAGES;
         const uint32_t round = it / C::NSTAGES;
-        if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1, p.timeout_ns, abort_flag, p.err, K_GEMV, 1)) {
-          ok = false;
-          break;
-        }
+        if (round > 0 && lane == 0)
+          ok = mbar_wait_bounded(&empty[s], (round - 1) & 1, p.timeout_ns, abort_flag, p.err, K_GEMV, 1);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
         uint8_t* st = smem + s * C::STAGE_BYTES;
-        const uint32_t bytes = static_cast<uint32_t>(nblk) * (32 * (TILE_N / 2) + ncols * 4 + ncols / 2) +
-                               static_cast<uint32_t>(mrows) * nblk * 128;
-        mbar_arrive_expect_tx(&full[s], bytes);
-        for (int j = 0; j < nblk; ++j) {
-          const int64_t b = blk + j;
-          tma_g2s_2d(st + j * 32 * (TILE_N / 2), &m.qw_map, t * (TILE_N / 2), static_cast<int32_t>(b * 32), &full[s]);
-          bulk_g2s(st + QW_STAGE + j * TILE_N * 4, m.scales + b * m.N + static_cast<int64_t>(t) * TILE_N,
-                   ncols * 4, &full[s]);
-          bulk_g2s(st + QW_STAGE + SC_STAGE + j * (TILE_N / 2),
-                   m.zp + (b * m.N + static_cast<int64_t>(t) * TILE_N) / 2, ncols / 2, &full[s]);
+        if (lane == 0) {
+          const uint32_t wbytes = full_stage ? static_cast<uint32_t>(QW_STAGE + SC_STAGE + ZP_STAGE)
+                                             : static_cast<uint32_t>(nblk) * (32 * (TILE_N / 2) + ncols * 4 + ncols / 2);
+          mbar_arrive_expect_tx(&full[s], wbytes + static_cast<uint32_t>(mrows) * nblk * 128);
         }
-        for (int r = 0; r < mrows; ++r)
-          bulk_g2s(st + QW_STAGE + SC_STAGE + ZP_STAGE + r * SB * 32 * 4,
-                   m.x + static_cast<int64_t>(mc * MT + r) * m.ldx + static_cast<int64_t>(blk) * 32, nblk * 128,
+        __syncwarp();
+        if (full_stage) {
+          if (lane == 0) tma_g2s_2d(st, &mp.qw_full, t * (TILE_N / 2), blk * 32, &full[s]);
+          if (lane == 1) tma_g2s_2d(st + QW_STAGE, &mp.sc_full, t * TILE_N, blk, &full[s]);
+          if (lane == 2) tma_g2s_2d(st + QW_STAGE + SC_STAGE, &mp.zp_full, t * (TILE_N / 2), blk, &full[s]);
+        } else if (lane < nblk) {
+          const int64_t b = blk + lane;
+          tma_g2s_2d(st + lane * 32 * (TILE_N / 2), &mp.qw_blk, t * (TILE_N / 2), static_cast<int32_t>(b * 32),
+                     &full[s]);
+          bulk_g2s(st + QW_STAGE + lane * TILE_N * 4, scol + b * m.N, ncols * 4, &full[s]);
+          bulk_g2s(st + QW_STAGE + SC_STAGE + lane * (TILE_N / 2), zcol + b * (m.N / 2), ncols / 2, &full[s]);
+        }
+        if (lane >= 8 && lane < 8 + mrows)
+          bulk_g2s(st + QW_STAGE + SC_STAGE + ZP_STAGE + (lane - 8) * SB * 32 * 4,
+                   xrow0 + static_cast<int64_t>(lane - 8) * m.ldx + static_cast<int64_t>(blk) * 32, nblk * 128,
                    &full[s]);
         ++it;
         blk += nblk;
-        cur += nblk;
       }
       f = seg_end;
     }
     // Copies still in flight must land before this CTA may exit: wait (bounded)
-    // for the last issued fill of every stage. In a normal run the consumers
-    // have already waited for all of them.
-    // Stage s was filled fills_s = ceil((it - s) / NSTAGES) times.
-    for (int s = 0; s < C::NSTAGES; ++s) {
-      const int fills_s = it > s ? (it - s + C::NSTAGES - 1) / C::NSTAGES : 0;
-      if (fills_s > 0) mbar_wait_bounded(&full[s], (fills_s - 1) & 1, p.timeout_ns, nullptr, p.err, K_GEMV, 2);
-    }
+    // for the last fill of every stage. In a normal run the consumers have
+    // already waited for all of them. Stage s was filled ceil((it - s) / NSTAGES)
+    // times.
+    if (lane == 0)
+      for (int s = 0; s < C::NSTAGES; ++s) {
+        const int fills_s = it > s ? (it - s + C::NSTAGES - 1) / C::NSTAGES : 0;
+        if (fills_s > 0) mbar_wait_bounded(&full[s], (fills_s - 1) & 1, p.timeout_ns, nullptr, p.err, K_GEMV, 2);
+      }
     return;
   }
 
@@ -207,9 +253,11 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
   bool ok = true;
 
   int64_t f = lo;
+  int g_hint = 0;
   while (f < hi) {
-    const Pos ps = locate(p, f);
-    const MatParams& m = p.mat[ps.g];
+    const Pos ps = locate(ms, p.count, f, g_hint);
+    g_hint = ps.g;
+    const MatScalars& m = ms[ps.g];
     const int64_t seg_end = min(hi, f + (m.nb - ps.blk));
     const int32_t t = static_cast<int32_t>(ps.tile_l / m.nmc);
     const int32_t mc = static_cast<int32_t>(ps.tile_l - static_cast<int64_t>(t) * m.nmc);
@@ -230,8 +278,10 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
       }
     }
 
-    for (int64_t cur = f; cur < seg_end; ) {
-      const int32_t nblk = static_cast<int32_t>(min(static_cast<int64_t>(SB), seg_end - cur));
+    int32_t blk = ps.blk;
+    const int32_t blk_end = blk + static_cast<int32_t>(seg_end - f);
+    while (blk < blk_end) {
+      const int32_t nblk = min(SB - (blk % SB), blk_end - blk);  // same grid as the producer
       const int s = it % C::NSTAGES;
       const uint32_t round = it / C::NSTAGES;
       if (ok) ok = mbar_wait_bounded(&full[s], round & 1, p.timeout_ns, abort_flag, p.err, K_GEMV, 3);
@@ -310,11 +360,10 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
       ++it;
-      cur += nblk;
+      blk += nblk;
     }
 
     // ---- segment done: reduce the NCW warps' partials, then write or fix up
-    const int32_t T = m.tile_off + static_cast<int32_t>(ps.tile_l);
     const int64_t t_start = f - ps.blk;
     const int64_t t_end = t_start + m.nb;
     const int64_t c_first = cta_of(t_start, p.W, G);
@@ -356,7 +405,7 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
     if (split) {
       __threadfence();
       named_bar_sync(1, C::NCW * 32);
-      if (ctid == 0) bcast[0] = ok ? atomicAdd(&p.ws_counters[T], 1) : -1;
+      if (ctid == 0) bcast[0] = ok ? atomicAdd(&p.ws_counters[c_first], 1) : -1;
       named_bar_sync(1, C::NCW * 32);
       const int prev = bcast[0];
       if (prev == static_cast<int>(c_last - c_first)) {
@@ -372,7 +421,7 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
             if (row < m.M && gcol < m.N) m.y[static_cast<int64_t>(row) * m.ldy + gcol] = v;
           }
         }
-        if (ctid == 0) p.ws_counters[T] = 0;
+        if (ctid == 0) p.ws_counters[c_first] = 0;
       }
       named_bar_sync(1, C::NCW * 32);
     }
@@ -418,15 +467,17 @@ Plan make_plan(const w4_desc* d, int count, int sms) {
     pl.total_tiles += static_cast<int32_t>(ntn * nmc);
     pl.W += ntn * nmc * (d[i].K / 32);
   }
-  pl.grid = static_cast<int>(std::min<int64_t>(sms, pl.W));
+  pl.grid = static_cast<int>(std::min<int64_t>(std::min(sms, 1024), pl.W));
   return pl;
 }
 
+// Workspace: [COUNTER_SLOTS int32 counters][grid][2][MT][TILE_N] fp32 partials.
+constexpr int COUNTER_SLOTS = 1024;  // >= grid (one per CTA)
+constexpr size_t COUNTER_BYTES = COUNTER_SLOTS * sizeof(int32_t);
+
 size_t ws_bytes(const Plan& pl) {
   if (pl.W == 0) return 0;
-  const size_t part = static_cast<size_t>(pl.grid) * 2 * pl.mt * TILE_N * sizeof(float);
-  const size_t cnt = static_cast<size_t>(pl.total_tiles) * sizeof(int32_t);
-  return part + ((cnt + 255) / 256) * 256;
+  return COUNTER_BYTES + static_cast<size_t>(pl.grid) * 2 * pl.mt * TILE_N * sizeof(float);
 }
 
 }  // namespace
@@ -460,7 +511,8 @@ w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cud
     return fail(W4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws == nullptr ? size_t(0) : ws_size);
   if ((reinterpret_cast<uintptr_t>(ws) & 15) != 0) return fail(W4_ERR_WORKSPACE, "workspace must be 16-byte aligned");
 
-  static thread_local GemvParams prm;  // ~12 KB: kept off the host stack
+  static_assert(sizeof(GemvParams) <= 32000, "kernel parameters must fit the 32 KB limit");
+  static thread_local GemvParams prm;  // ~31 KB: kept off the host stack
   std::memset(&prm, 0, sizeof(prm));
   int g = 0;
   int64_t bt = 0;
@@ -468,9 +520,11 @@ w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cud
   for (int i = 0; i < count; ++i) {
     const w4_desc& s = d[i];
     if (s.M == 0 || s.N == 0 || s.K == 0) continue;
-    MatParams& m = prm.mat[g];
-    w4_status rc = encode_qw_map(&m.qw_map, s.qw, s.K, s.N);
+    MatParams& mpar = prm.mat[g];
+    w4_status rc = encode_w4_maps(&mpar.qw_full, &mpar.qw_blk, &mpar.sc_full, &mpar.zp_full, s.qw, s.scales, s.zp,
+                                  s.K, s.N);
     if (rc != W4_OK) return rc;
+    MatScalars& m = mpar.s;
     m.x = s.x;
     m.scales = s.scales;
     m.zp = s.zp;
@@ -483,7 +537,6 @@ w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cud
     m.nb = static_cast<int32_t>(s.K / 32);
     m.ntn = static_cast<int32_t>((s.N + TILE_N - 1) / TILE_N);
     m.nmc = static_cast<int32_t>((s.M + pl.mt - 1) / pl.mt);
-    m.tile_off = tiles;
     m.bt_off = bt;
     tiles += m.ntn * m.nmc;
     bt += static_cast<int64_t>(m.ntn) * m.nmc * m.nb;
@@ -492,9 +545,8 @@ w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cud
   prm.count = g;
   prm.W = bt;
   prm.total_tiles = tiles;
-  prm.ws_partials = static_cast<float*>(ws);
-  prm.ws_counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) +
-                                               static_cast<size_t>(pl.grid) * 2 * pl.mt * TILE_N * sizeof(float));
+  prm.ws_counters = static_cast<int32_t*>(ws);
+  prm.ws_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + COUNTER_BYTES);
   prm.err = di.err;
   prm.timeout_ns = wait_timeout_ns();
   switch (pl.mt) {

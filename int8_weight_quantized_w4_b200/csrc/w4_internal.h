@@ -33,8 +33,11 @@ w4_status fail(w4_status s, const char* fmt, ...);
 w4_status cuda_fail(cudaError_t e, const char* what);
 uint64_t wait_timeout_ns();
 
-// Tensor map of a [K rows][N/2 bytes] nibble matrix, box 32 rows x 128 bytes.
-w4_status encode_qw_map(CUtensorMap* map, const uint8_t* qw, int64_t K, int64_t N);
+// Tensor maps of one packed weight: nibbles [K][N/2 B] with boxes of 256 and
+// 32 rows x 128 B, scales [K/32][N] fp32 with box 8 x 256, zero points
+// [K/32][N/2 B] with box 8 x 128 B. Cached per (pointers, K, N).
+w4_status encode_w4_maps(CUtensorMap* qw_full, CUtensorMap* qw_blk, CUtensorMap* sc_full, CUtensorMap* zp_full,
+                         const uint8_t* qw, const float* scales, const uint8_t* zp, int64_t K, int64_t N);
 
 // ---- body kernels
 bool gemv_eligible(const w4_desc& d, const char** why);
@@ -55,7 +58,8 @@ struct HeadArgs {
   int64_t ldl;
   int64_t M, K, V;
 };
-w4_status launch_head(const HeadArgs& a, cudaStream_t st, const DeviceInfo& di);
+size_t head_workspace_bytes(int64_t M, int64_t K, int64_t V, int sms);
+w4_status launch_head(const HeadArgs& a, void* ws, size_t ws_size, cudaStream_t st, const DeviceInfo& di);
 w4_status launch_head_generic(const HeadArgs& a, cudaStream_t st, const DeviceInfo& di);
 
 // ---- diagnostics

@@ -106,7 +106,7 @@ def test_head_argument_errors(kw, status):
     a = dict(h=0x1000, ldh=32, table=0x2000, ldt=20, scales=0x3000, logits=0x4000, ldl=20, M=1, K=32, V=20)
     a.update(kw)
     st = lib.i8_head_logits(a["h"], a["ldh"], a["table"], a["ldt"], a["scales"], a["logits"], a["ldl"], a["M"],
-                            a["K"], a["V"], None)
+                            a["K"], a["V"], None, 0, None)
     assert st == status
 
 

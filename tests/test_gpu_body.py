@@ -140,6 +140,22 @@ def test_deterministic():
     assert torch().equal(y1, y2)
 
 
+def test_workspace_reused_across_shapes():
+    """One workspace through calls whose grids and split tiles differ: the
+    counters must be back at zero after every call."""
+    T = torch()
+    ws = T.zeros(1 << 22, dtype=T.uint8, device="cuda")
+    for (M, K, N) in [(1, 768, 768), (1, 64, 288), (3, 3072, 768), (1, 64, 288), (8, 96, 544), (1, 8192, 64)]:
+        W = synth.w4_weight(K, N, 77)
+        x = synth.activations(M, K, 77)
+        Wd = upload_w4(W)
+        y = w4().w4_matmul(dev(x), Wd["qw"], Wd["scales"], Wd["zp"], K, N, path="gemv", ws=ws)
+        T.cuda.synchronize()
+        y_ref, a = oracle.w4_matmul_ref(x, W["qw"], W["scales"], W["zp"], K, N)
+        check(y, y_ref, a, f"reuse M={M} K={K} N={N}")
+    assert int(ws[:4096].count_nonzero()) == 0
+
+
 def test_workspace_too_small_is_refused():
     T = torch()
     K, N = 768, 768
