@@ -129,6 +129,28 @@ W4_API w4_status w4_matmul_path(const float* x, int64_t ldx, const uint8_t* qw, 
                          int64_t N, void* workspace, size_t workspace_bytes, w4_path path,
                          void* stream);
 
+/* Allocation-free form of w4_matmul. The pages describe no such entry point;
+ * it exists for callers that cannot allocate device memory where they
+ * multiply (for example a plugin inside a framework that owns every device
+ * allocation, or a process that forbids allocation after start-up). Inputs
+ * and outputs are the caller's, exactly as for w4_matmul; the split-K scratch
+ * comes from one array of W4_NOALLOC_SCRATCH_BYTES inside this library,
+ * which every GPU that loads the library keeps until the process exits.
+ * - Shapes whose scratch need (w4_matmul_workspace_size) exceeds that size
+ *   are refused with W4_ERR_WORKSPACE. The need grows with M and with the
+ *   number of SMs the call keeps busy: on a 148-SM B200 every M <= 4 fits,
+ *   and M from 5 to 16 fits only for weights too small to fill the GPU.
+ * - Each call clears the part of the array it uses, then runs as w4_matmul.
+ *   Calls share the array, so calls that overlap on the GPU (other streams,
+ *   other host threads on the same device) race: serialise them.
+ * - The first call on a device looks up the array's device address; make
+ *   that first call before any stream capture.
+ * Calls no allocating routine. */
+#define W4_NOALLOC_SCRATCH_BYTES (2u << 20)
+W4_API w4_status w4_matmul_noalloc(const float* x, int64_t ldx, const uint8_t* qw, const float* scales,
+                                   const uint8_t* zp, float* y, int64_t ldy, int64_t M, int64_t K,
+                                   int64_t N, void* stream);
+
 /* Many independent matmuls (for example the 48 weights of a decoder stack)
  * in as few launches as possible: up to W4_GROUP_MAX descriptors share one
  * persistent launch whose work is split evenly over the SMs. `descs` is a
