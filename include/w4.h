@@ -146,7 +146,7 @@ W4_API w4_status w4_matmul_path(const float* x, int64_t ldx, const uint8_t* qw, 
  * - The first call on a device looks up the array's device address; make
  *   that first call before any stream capture.
  * Calls no allocating routine. */
-#define W4_NOALLOC_SCRATCH_BYTES (2u << 20)
+#define W4_NOALLOC_SCRATCH_BYTES (4u << 20)
 W4_API w4_status w4_matmul_noalloc(const float* x, int64_t ldx, const uint8_t* qw, const float* scales,
                                    const uint8_t* zp, float* y, int64_t ldy, int64_t M, int64_t K,
                                    int64_t N, void* stream);

@@ -16,8 +16,8 @@
 //    position c + r_w of warp w). A tile is 31 chunks wide, so every warp's
 //    32-chunk window covers it whatever r_w is.
 //  * int8 -> fp32 exactly with one PRMT per element: the byte, biased by
-//    0x80, is placed in the mantissa of 2^23 (0x4B0000uu), then one packed
-//    f32x2 add removes 2^23 + 128. The per-token scale is applied once per
+//    0x80, is placed in the mantissa of 2^23 (0x4B0000uu), then one FADD
+//    removes 2^23 + 128. The per-token scale is applied once per
 //    column after the sum.
 //  * Persistent stream-K, like the W4 GEMV: the units (16-row group of one
 //    column tile of one group of MT rows of h) form one flat range split
@@ -51,9 +51,18 @@ struct HCfg {
   static constexpr int SMEM = RED_FLOATS * 4 + NW * 4 + 16;
 };
 
-__device__ __forceinline__ float byte_magic(uint32_t biased_word, int j) {
-  // bytes of the result: [biased byte j, 0x00, 0x00, 0x4B]
-  return __uint_as_float(__byte_perm(biased_word, 0x4B000000u, 0x7540u + j));
+// One PRMT: bytes of the result are [biased byte j, 0x00, 0x00, 0x4B]; the
+// 0x4B000000 word is passed in a register so the selector is the only
+// immediate.
+__device__ __forceinline__ float byte_magic(uint32_t biased_word, uint32_t magic, int j /*compile time*/) {
+  uint32_t r;
+  switch (j) {
+    case 0: asm("prmt.b32 %0, %1, %2, 0x7540;" : "=r"(r) : "r"(biased_word), "r"(magic)); break;
+    case 1: asm("prmt.b32 %0, %1, %2, 0x7541;" : "=r"(r) : "r"(biased_word), "r"(magic)); break;
+    case 2: asm("prmt.b32 %0, %1, %2, 0x7542;" : "=r"(r) : "r"(biased_word), "r"(magic)); break;
+    default: asm("prmt.b32 %0, %1, %2, 0x7543;" : "=r"(r) : "r"(biased_word), "r"(magic)); break;
+  }
+  return __uint_as_float(r);
 }
 
 template <int CB>
@@ -128,7 +137,8 @@ __global__ void __launch_bounds__(NW * 32, HCfg<MT>::MINB) i8_head_kernel(const 
   const int64_t lo = range_lo(blockIdx.x, p.U, G);
   const int64_t hi = range_lo(blockIdx.x + 1, p.U, G);
   const int8_t* table_end = p.table + (static_cast<int64_t>(p.K) - 1) * p.ldt + p.V;
-  const float2 bias = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
+  uint32_t kMagic;  // 0x4B000000 (the bits of 2^23) held in a register
+  asm("mov.b32 %0, 0x4B000000;" : "=r"(kMagic));
 
   int64_t f = lo;
   while (f < hi) {
@@ -204,13 +214,13 @@ __global__ void __launch_bounds__(NW * 32, HCfg<MT>::MINB) i8_head_kernel(const 
         for (int i = 0; i < CB / 4; ++i) {
           const uint32_t bw = cur[j].w[i] ^ 0x80808080u;
 #pragma unroll
-          for (int pr = 0; pr < 2; ++pr) {
-            const float2 e = make_float2(byte_magic(bw, 2 * pr), byte_magic(bw, 2 * pr + 1));
-            const float2 qv = __fadd2_rn(e, bias);  // exact int8 values
+          for (int e = 0; e < 4; ++e) {
+            const float qv = byte_magic(bw, kMagic, e) - 8388736.0f;  // exact int8 value
 #pragma unroll
             for (int mm = 0; mm < MT; ++mm) {
-              const float2 hh = make_float2(hcur[j][mm], hcur[j][mm]);
-              acc[mm * (CB / 2) + i * 2 + pr] = __ffma2_rn(hh, qv, acc[mm * (CB / 2) + i * 2 + pr]);
+              float2& a2 = acc[mm * (CB / 2) + i * 2 + (e >> 1)];
+              if (e & 1) a2.y = fmaf(hcur[j][mm], qv, a2.y);
+              else a2.x = fmaf(hcur[j][mm], qv, a2.x);
             }
           }
         }

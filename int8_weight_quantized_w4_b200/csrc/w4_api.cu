@@ -111,18 +111,12 @@ static w4_status encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void*
 namespace {
 struct MapKey {
   const void* qw;
-  const void* sc;
-  const void* zp;
   int64_t K, N;
-  bool operator==(const MapKey& o) const {
-    return qw == o.qw && sc == o.sc && zp == o.zp && K == o.K && N == o.N;
-  }
+  bool operator==(const MapKey& o) const { return qw == o.qw && K == o.K && N == o.N; }
 };
 struct MapKeyHash {
   size_t operator()(const MapKey& k) const {
     size_t h = reinterpret_cast<size_t>(k.qw) * 0x9E3779B97F4A7C15ull;
-    h ^= reinterpret_cast<size_t>(k.sc) + 0x7F4A7C159E3779B9ull + (h << 6) + (h >> 2);
-    h ^= reinterpret_cast<size_t>(k.zp) + (h << 6) + (h >> 2);
     h ^= static_cast<size_t>(k.K) * 31 + static_cast<size_t>(k.N) + (h << 6) + (h >> 2);
     return h;
   }
@@ -135,21 +129,23 @@ std::unordered_map<MapKey, MapSet, MapKeyHash> g_map_cache;
 constexpr size_t kMapCacheMax = 4096;
 }  // namespace
 
-// The four tensor maps of one packed weight (the GEMV's copies). A map is a
-// pure function of (pointers, K, N), so the cache can never return a stale
-// one: reusing freed memory for another weight of the same shape yields the
-// same map.
-w4_status encode_w4_maps(CUtensorMap* qw_full, CUtensorMap* qw_blk, CUtensorMap* sc_full, CUtensorMap* zp_full,
-                         const uint8_t* qw, const float* scales, const uint8_t* zp, int64_t K, int64_t N) {
-  const MapKey key{qw, scales, zp, K, N};
+// The four tensor maps of one packed weight, all over the [K rows][N/2 bytes]
+// nibble matrix: 256-byte-wide boxes of 128 and 16 rows (wide tiles) and
+// 128-byte-wide boxes of 256 and 32 rows (narrow tiles). A map is a pure
+// function of (pointer, K, N), so the cache can never return a stale one:
+// reusing freed memory for another weight of the same shape yields the same
+// map.
+w4_status encode_w4_maps(CUtensorMap* wide_full, CUtensorMap* wide_unit, CUtensorMap* narrow_full,
+                         CUtensorMap* narrow_unit, const uint8_t* qw, int64_t K, int64_t N) {
+  const MapKey key{qw, K, N};
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto itc = g_map_cache.find(key);
     if (itc != g_map_cache.end()) {
-      *qw_full = itc->second.m[0];
-      *qw_blk = itc->second.m[1];
-      *sc_full = itc->second.m[2];
-      *zp_full = itc->second.m[3];
+      *wide_full = itc->second.m[0];
+      *wide_unit = itc->second.m[1];
+      *narrow_full = itc->second.m[2];
+      *narrow_unit = itc->second.m[3];
       return W4_OK;
     }
   }
@@ -162,17 +158,17 @@ w4_status encode_w4_maps(CUtensorMap* qw_full, CUtensorMap* qw_blk, CUtensorMap*
       g_encode = reinterpret_cast<EncodeTiledFn>(fn);
   });
   if (g_encode == nullptr) return fail(W4_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const uint64_t half = static_cast<uint64_t>(N / 2), nb = static_cast<uint64_t>(K / 32);
+  const uint64_t half = static_cast<uint64_t>(N / 2);
   MapSet ms;
   w4_status rc;
-  if ((rc = encode_2d(&ms.m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, half, K, half, 128, 256)) != W4_OK) return rc;
-  if ((rc = encode_2d(&ms.m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, half, K, half, 128, 32)) != W4_OK) return rc;
-  if ((rc = encode_2d(&ms.m[2], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, scales, N, nb, N * 4, 256, 8)) != W4_OK) return rc;
-  if ((rc = encode_2d(&ms.m[3], CU_TENSOR_MAP_DATA_TYPE_UINT8, zp, half, nb, half, 128, 8)) != W4_OK) return rc;
-  *qw_full = ms.m[0];
-  *qw_blk = ms.m[1];
-  *sc_full = ms.m[2];
-  *zp_full = ms.m[3];
+  if ((rc = encode_2d(&ms.m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, half, K, half, 256, 128)) != W4_OK) return rc;
+  if ((rc = encode_2d(&ms.m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, half, K, half, 256, 16)) != W4_OK) return rc;
+  if ((rc = encode_2d(&ms.m[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, half, K, half, 128, 256)) != W4_OK) return rc;
+  if ((rc = encode_2d(&ms.m[3], CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, half, K, half, 128, 32)) != W4_OK) return rc;
+  *wide_full = ms.m[0];
+  *wide_unit = ms.m[1];
+  *narrow_full = ms.m[2];
+  *narrow_unit = ms.m[3];
   std::lock_guard<std::mutex> lk(g_map_mu);
   if (g_map_cache.size() >= kMapCacheMax) g_map_cache.clear();
   g_map_cache.emplace(key, ms);

@@ -75,32 +75,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended (it issues nothing) until the phase completes or about hint_ns
+// pass, instead of spinning and taking issue slots from working warps.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with parity `parity` of `bar` has completed. Returns
 // false (after recording the error) when `timeout_ns` passes first, or when
-// *abort is set by another thread of the CTA. The timer and the abort flag
-// are looked at once every 1024 polls, so a waiting warp costs few issue
-// slots (try_wait itself suspends the thread for a while when the phase is
-// not complete).
+// *abort is set by another thread of the CTA. Each try suspends the thread
+// for up to 0.2 ms, so a waiting warp costs almost no issue slots and the
+// timer and the abort flag are looked at after every try.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
                                                   volatile int* abort, ErrorWord* err, int32_t kernel,
                                                   int32_t detail) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
-  uint64_t t0 = 0;
-  uint32_t n = 0;
+  const uint64_t t0 = globaltimer_ns();
 #pragma unroll 1
   while (true) {
-    if (mbar_try_wait(a, parity)) return true;
-    if ((++n & 1023u) == 0) {
-      if (abort != nullptr && *abort) return false;
-      const uint64_t t = globaltimer_ns();
-      if (t0 == 0) {
-        t0 = t;
-      } else if (t - t0 > timeout_ns) {
-        if (abort != nullptr) *abort = 1;
-        record_error(err, W4_ERR_TIMEOUT, kernel, detail);
-        return false;
-      }
+    if (mbar_try_wait_sleep(a, parity, 200000u)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      if (abort != nullptr) *abort = 1;
+      record_error(err, W4_ERR_TIMEOUT, kernel, detail);
+      return false;
     }
   }
 }
@@ -148,6 +156,19 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 // built the same way from the zero-point word gives (q - zp) * 16^(i mod 4)
 // exactly: both operands are integers in [2^23, 2^24). The power of two is
 // folded into the scale, s * 16^-(i mod 4), which is exact too.
+
+// One LOP3: (word & mask) | magic, with the magic exponent word passed in a
+// register so that the instruction needs only one immediate (the mask).
+__device__ __forceinline__ float magic_nib_r(uint32_t word, uint32_t magic, int slot /*0..3, compile time*/) {
+  uint32_t r;
+  switch (slot) {
+    case 0: asm("lop3.b32 %0, %1, 0xF, %2, 0xEA;" : "=r"(r) : "r"(word), "r"(magic)); break;
+    case 1: asm("lop3.b32 %0, %1, 0xF0, %2, 0xEA;" : "=r"(r) : "r"(word), "r"(magic)); break;
+    case 2: asm("lop3.b32 %0, %1, 0xF00, %2, 0xEA;" : "=r"(r) : "r"(word), "r"(magic)); break;
+    default: asm("lop3.b32 %0, %1, 0xF000, %2, 0xEA;" : "=r"(r) : "r"(word), "r"(magic)); break;
+  }
+  return __uint_as_float(r);
+}
 
 __device__ __forceinline__ float magic_nib(uint32_t word, int slot /*0..3*/) {
   return __uint_as_float(0x4B000000u | (word & (0xFu << (4 * slot))));

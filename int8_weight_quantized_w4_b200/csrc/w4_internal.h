@@ -33,11 +33,11 @@ w4_status fail(w4_status s, const char* fmt, ...);
 w4_status cuda_fail(cudaError_t e, const char* what);
 uint64_t wait_timeout_ns();
 
-// Tensor maps of one packed weight: nibbles [K][N/2 B] with boxes of 256 and
-// 32 rows x 128 B, scales [K/32][N] fp32 with box 8 x 256, zero points
-// [K/32][N/2 B] with box 8 x 128 B. Cached per (pointers, K, N).
-w4_status encode_w4_maps(CUtensorMap* qw_full, CUtensorMap* qw_blk, CUtensorMap* sc_full, CUtensorMap* zp_full,
-                         const uint8_t* qw, const float* scales, const uint8_t* zp, int64_t K, int64_t N);
+// Tensor maps of one packed weight's nibbles [K rows][N/2 bytes]: boxes of
+// 128 and 16 rows x 256 B (wide tiles), 256 and 32 rows x 128 B (narrow
+// tiles). Cached per (pointer, K, N).
+w4_status encode_w4_maps(CUtensorMap* wide_full, CUtensorMap* wide_unit, CUtensorMap* narrow_full,
+                         CUtensorMap* narrow_unit, const uint8_t* qw, int64_t K, int64_t N);
 
 // ---- body kernels
 bool gemv_eligible(const w4_desc& d, const char** why);
