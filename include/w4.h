@@ -138,15 +138,17 @@ W4_API w4_status w4_matmul_path(const float* x, int64_t ldx, const uint8_t* qw, 
  * which every GPU that loads the library keeps until the process exits.
  * - Shapes whose scratch need (w4_matmul_workspace_size) exceeds that size
  *   are refused with W4_ERR_WORKSPACE. The need grows with M and with the
- *   number of SMs the call keeps busy: on a 148-SM B200 every M <= 4 fits,
- *   and M from 5 to 16 fits only for weights too small to fill the GPU.
+ *   number of SMs the call keeps busy (4 KB + SMs x M' x 4 KB, M' = M
+ *   rounded up to 1, 2, 4 or 8): on a 148-SM B200 every M <= 2 fits (at
+ *   most 1.2 MB), while M from 3 to 16 fits only for weights too small to
+ *   fill the GPU.
  * - Each call clears the part of the array it uses, then runs as w4_matmul.
  *   Calls share the array, so calls that overlap on the GPU (other streams,
  *   other host threads on the same device) race: serialise them.
  * - The first call on a device looks up the array's device address; make
  *   that first call before any stream capture.
  * Calls no allocating routine. */
-#define W4_NOALLOC_SCRATCH_BYTES (4u << 20)
+#define W4_NOALLOC_SCRATCH_BYTES (2u << 20)
 W4_API w4_status w4_matmul_noalloc(const float* x, int64_t ldx, const uint8_t* qw, const float* scales,
                                    const uint8_t* zp, float* y, int64_t ldy, int64_t M, int64_t K,
                                    int64_t N, void* stream);

@@ -34,7 +34,7 @@ def test_noalloc_matches_w4_matmul_on_two_calls_in_a_row():
     import int8_weight_quantized_w4_b200 as w4
     lib = w4.lib()
     stream = torch.cuda.current_stream().cuda_stream
-    cases = [(1, 768, 3072, 901), (4, 3072, 768, 902)]
+    cases = [(1, 768, 3072, 901), (2, 3072, 768, 902)]
     host, dev, got = [], [], []
     for M, K, N, tag in cases:
         W = synth.w4_weight(K, N, tag)
@@ -63,7 +63,7 @@ def test_noalloc_refuses_shapes_beyond_its_scratch():
     import int8_weight_quantized_w4_b200 as w4
     lib = w4.lib()
     M, K, N = 8, 3072, 768  # enough work to use every SM
-    assert w4.w4_matmul_workspace_size(M, K, N) > 4 << 20
+    assert w4.w4_matmul_workspace_size(M, K, N) > 2 << 20
     W = synth.w4_weight(K, N, 903)
     Wd = {k: torch.from_numpy(W[k]).cuda() for k in ("qw", "scales", "zp")}
     xd = torch.from_numpy(synth.activations(M, K, 903)).cuda()
