@@ -4,27 +4,37 @@
 // scale per token, [768, V] layout) and 4 (last_token_logits: only the last
 // position's rows h are multiplied).
 //
-// Design (sm_100a):
-//  * Row k of T starts at byte k*ldt, which is not aligned when ldt is odd
-//    (V = 50257). With T 16-byte aligned, (k*ldt) mod 16 depends only on
-//    k mod 16, so a warp that takes the rows k = 16 g + w (w = warp, g a
-//    16-row group) sees ONE misalignment r_w for all its rows. Each lane then
-//    loads aligned CB-byte chunks (LDG.128 for CB = 16) and the warp's 32
-//    lanes cover the byte window that starts r_w bytes before the tile's
-//    first column: no realignment in registers at all. The reduction across
-//    warps undoes the per-warp shift (column c of the tile sits at window
-//    position c + r_w of warp w). A tile is 31 chunks wide, so every warp's
-//    32-chunk window covers it whatever r_w is.
-//  * int8 -> fp32 exactly with one PRMT per element: the byte, biased by
-//    0x80, is placed in the mantissa of 2^23 (0x4B0000uu), then one FADD
-//    removes 2^23 + 128. The per-token scale is applied once per
-//    column after the sum.
-//  * Persistent stream-K, like the W4 GEMV: the units (16-row group of one
-//    column tile of one group of MT rows of h) form one flat range split
-//    evenly over the CTAs (one per SM). Each warp keeps the loads of the
-//    next D rows in flight while it converts and accumulates the current D. A tile whose rows straddle CTAs is finished by the last
-//    CTA to arrive, which adds the partials in CTA order (deterministic)
-//    through the caller's workspace and resets the counter to zero.
+// Two kernels share the exact int8 -> fp32 decode: the byte, biased by 0x80,
+// is placed in the mantissa of 2^23 (0x4B0000uu) by one PRMT, then one
+// subtraction removes 2^23 + 128. The per-token scale is applied once per
+// column after the sum.
+//
+// Row k of T starts at byte k*ldt, which is not aligned when ldt is odd
+// (V = 50257). With T 16-byte aligned, (k*ldt) mod 16 depends only on
+// k mod 16, so the rows k = 16 g + j (one residue j) share ONE misalignment:
+// a thread that reads aligned 16-byte chunks of only those rows sees every
+// column at the same place in its chunk, and the reduction across residues
+// undoes the per-residue shift.
+//
+// i8_rows_kernel (M <= 2): one column slice of at most 368 columns per CTA
+// and all K rows of it, so no CTA shares a tile with another. Thread
+// (chunk c of 24, residue j of 16) copies, with 16-byte asynchronous copies,
+// chunk c of the 16-byte-aligned window around the slice of each of its rows
+// (k = j mod 16) into its own shared-memory slot, six stages of four rows
+// ahead of the ones it converts (the copy holding the table's last byte reads
+// only up to it and zero-fills the rest). It converts rows k and k + 16
+// together, so the subtraction and the FMA are packed f32x2 instructions with
+// h[k], h[k+16] as one operand. At the end the 16 residues' column sums are
+// added with their shifts undone. No thread waits on another except at that
+// final reduction.
+//
+// i8_head_kernel (M >= 3): persistent stream-K over 16-row groups of narrow
+// column tiles. A warp takes one row of every 16-row group (one residue);
+// each lane loads aligned chunks of it, keeping the loads of the next D rows
+// in flight while it converts and accumulates the current D. A tile whose
+// rows straddle CTAs is finished by the last CTA to arrive, which adds the
+// partials in CTA order (deterministic) through the caller's workspace and
+// resets the counter to zero.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -293,6 +303,199 @@ __global__ void __launch_bounds__(NW * 32, HCfg<MT>::MINB) i8_head_kernel(const 
   }
 }
 
+// ---------------------------------------------------------------- i8_rows_kernel
+
+constexpr int RROWS = 64;             // rows per stage
+constexpr int RWIN = 384;             // window bytes per row (24 chunks of 16 B)
+constexpr int RTV = RWIN - 16;        // columns a slice may hold (any shift fits)
+constexpr int RST = 6;                // stages in flight per thread
+constexpr int RTHREADS = 384;         // 24 chunks x 16 residues
+constexpr int RSTAGE = RROWS * RWIN;  // 24 KB
+constexpr int RH_MAX_BYTES = 32768;   // h rows kept in shared memory
+
+struct RowsParams {
+  const float* h;
+  int64_t ldh;
+  const int8_t* table;
+  int64_t ldt;
+  const float* scales;
+  float* logits;
+  int64_t ldl;
+  int32_t M, K, V;
+  int32_t ntiles;  // column slices, [t*V/ntiles, (t+1)*V/ntiles)
+  int32_t kpad;    // K rounded up to whole stages
+  int32_t pad;
+};
+
+template <int MT>
+size_t rows_smem_bytes(int kpad) {
+  return static_cast<size_t>(RST) * RSTAGE + static_cast<size_t>(MT) * 16 * RWIN * 4 +
+         static_cast<size_t>(MT) * kpad * 4 + 64;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(RTHREADS, 1) i8_rows_kernel(const __grid_constant__ RowsParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  float* red = reinterpret_cast<float*>(smem + RST * RSTAGE);  // [MT][16 residues][RWIN]
+  float* hs = red + MT * 16 * RWIN;                            // [MT][kpad], zero past K
+  int* shifts = reinterpret_cast<int*>(hs + MT * p.kpad);      // [16]
+
+  const int t = threadIdx.x;
+  const int ch = t % 24;   // 16-byte chunk of the row window
+  const int res = t / 24;  // residue of this thread's rows mod 16
+  const int nst = p.kpad / RROWS;
+  const uintptr_t tend = reinterpret_cast<uintptr_t>(p.table + static_cast<int64_t>(p.K - 1) * p.ldt + p.V);
+  const int64_t step16 = 16 * p.ldt;  // from row k to row k + 16
+  uint32_t kMagic;                    // 0x4B000000 (the bits of 2^23) held in a register
+  asm("mov.b32 %0, 0x4B000000;" : "=r"(kMagic));
+  const float2 kOff = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
+
+  for (int i = t; i < MT * p.kpad; i += RTHREADS) {
+    const int mm = i / p.kpad, k = i - mm * p.kpad;
+    hs[i] = (mm < p.M && k < p.K) ? p.h[static_cast<int64_t>(mm) * p.ldh + k] : 0.f;
+  }
+  __syncthreads();
+
+  for (int tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x) {
+    const int64_t v0 = static_cast<int64_t>(tile) * p.V / p.ntiles;
+    const int64_t v1 = static_cast<int64_t>(tile + 1) * p.V / p.ntiles;
+    const int ncols = static_cast<int>(v1 - v0);
+    // This thread's chunk of row k = res + 16 j is at a0 + j * step16; it is
+    // part of the row's window iff 16 ch < (window end - window start), the
+    // same for every row of the residue.
+    const uintptr_t x0 = reinterpret_cast<uintptr_t>(p.table + static_cast<int64_t>(res) * p.ldt + v0);
+    const uintptr_t a0 = (x0 & ~static_cast<uintptr_t>(15)) + 16 * ch;
+    const bool active = a0 < x0 + static_cast<uintptr_t>(ncols);
+    uint8_t* mine = smem + t * 16;  // this thread's slot: [stage][row q][thread] of 16 B
+
+    // stage sg holds this thread's rows k = 64 sg + res + 16 q, q = 0..3
+    auto issue = [&](int sg) {
+      if (sg < nst && active) {
+        uint8_t* dst = mine + (sg % RST) * RSTAGE;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int k = sg * RROWS + res + 16 * q;
+          if (k < p.K) {
+            const uintptr_t src = a0 + static_cast<uintptr_t>(4 * sg + q) * static_cast<uintptr_t>(step16);
+            const uint32_t n = tend - src >= 16 ? 16u : static_cast<uint32_t>(tend - src);  // rest zero-filled
+            cp_async_16(dst + q * RTHREADS * 16, reinterpret_cast<const void*>(src), n);
+          }
+        }
+      }
+      cp_async_commit();
+    };
+
+    float2 acc[MT][16];
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) acc[mm][c] = make_float2(0.f, 0.f);
+#pragma unroll 1
+    for (int sg = 0; sg < RST - 1; ++sg) issue(sg);
+#pragma unroll 1
+    for (int sg = 0; sg < nst; ++sg) {
+      issue(sg + RST - 1);
+      cp_async_wait_group<RST - 1>();  // this thread's copies of stage sg have landed
+      const uint8_t* src = mine + (sg % RST) * RSTAGE;
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        // rows k and k + 16 (q = 2 pr and 2 pr + 1), both residue res
+        const uint4 A = *reinterpret_cast<const uint4*>(src + (2 * pr) * RTHREADS * 16);
+        const uint4 B = *reinterpret_cast<const uint4*>(src + (2 * pr + 1) * RTHREADS * 16);
+        const int k0 = sg * RROWS + res + 32 * pr;
+        float2 hp[MT];
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm) hp[mm] = make_float2(hs[mm * p.kpad + k0], hs[mm * p.kpad + k0 + 16]);
+        const uint32_t wa[4] = {A.x, A.y, A.z, A.w};
+        const uint32_t wb[4] = {B.x, B.y, B.z, B.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t a = wa[i] ^ 0x80808080u;
+          const uint32_t b = wb[i] ^ 0x80808080u;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 d = __fadd2_rn(make_float2(byte_magic(a, kMagic, e), byte_magic(b, kMagic, e)), kOff);
+#pragma unroll
+            for (int mm = 0; mm < MT; ++mm) acc[mm][i * 4 + e] = __ffma2_rn(hp[mm], d, acc[mm][i * 4 + e]);
+          }
+        }
+      }
+    }
+    cp_async_wait_group<0>();
+    // ---- reduce the residues: column c of the slice sits at byte c + shift[j]
+    // of residue j's window
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm) {
+      float* dst = red + (mm * 16 + res) * RWIN + ch * 16;
+#pragma unroll
+      for (int c = 0; c < 16; c += 4)
+        *reinterpret_cast<float4*>(dst + c) =
+            make_float4(acc[mm][c].x + acc[mm][c].y, acc[mm][c + 1].x + acc[mm][c + 1].y,
+                        acc[mm][c + 2].x + acc[mm][c + 2].y, acc[mm][c + 3].x + acc[mm][c + 3].y);
+    }
+    if (t < 16)
+      shifts[t] = static_cast<int>(reinterpret_cast<uintptr_t>(p.table + static_cast<int64_t>(t) * p.ldt + v0) & 15);
+    __syncthreads();
+    for (int c = t; c < ncols; c += RTHREADS) {
+      const float sc = __ldg(p.scales + v0 + c);
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        if (mm >= p.M) break;
+        float v = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v += red[(mm * 16 + j) * RWIN + c + shifts[j]];
+        p.logits[static_cast<int64_t>(mm) * p.ldl + v0 + c] = v * sc;
+      }
+    }
+    __syncthreads();  // red and shifts are reused by the next slice
+  }
+}
+
+template <int MT>
+w4_status launch_rows_mt(const RowsParams& prm, int grid, cudaStream_t st, const w4host::DeviceInfo& di) {
+  const size_t smem = rows_smem_bytes<MT>(prm.kpad);
+  static size_t configured[64] = {};
+  if (di.dev < 64 && configured[di.dev] < smem) {
+    cudaError_t e = cudaFuncSetAttribute(i8_rows_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return w4host::cuda_fail(e, "cudaFuncSetAttribute(i8_rows)");
+    configured[di.dev] = smem;
+  }
+  i8_rows_kernel<MT><<<grid, RTHREADS, smem, st>>>(prm);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W4_OK : w4host::cuda_fail(e, "launch i8_rows");
+}
+
+// The rows kernel takes M <= 2 while h fits its shared-memory copy.
+bool rows_eligible(int64_t M, int64_t K) {
+  const int64_t kpad = (K + RROWS - 1) / RROWS * RROWS;
+  return M <= 2 && M * kpad * 4 <= RH_MAX_BYTES;
+}
+
+w4_status launch_rows(const w4host::HeadArgs& a, cudaStream_t st, const w4host::DeviceInfo& di) {
+  RowsParams prm;
+  prm.h = a.h;
+  prm.ldh = a.ldh;
+  prm.table = a.table;
+  prm.ldt = a.ldt;
+  prm.scales = a.scales;
+  prm.logits = a.logits;
+  prm.ldl = a.ldl;
+  prm.M = static_cast<int32_t>(a.M);
+  prm.K = static_cast<int32_t>(a.K);
+  prm.V = static_cast<int32_t>(a.V);
+  prm.kpad = static_cast<int32_t>((a.K + RROWS - 1) / RROWS * RROWS);
+  prm.pad = 0;
+  // slices of at most RTV columns, at least one per SM when V allows 32-column
+  // slices, and a whole number of rounds over the SMs
+  int64_t nt = (a.V + RTV - 1) / RTV;
+  nt = std::max<int64_t>(nt, std::min<int64_t>(di.sms, (a.V + 31) / 32));
+  if (nt > di.sms) nt = (nt + di.sms - 1) / di.sms * di.sms;
+  prm.ntiles = static_cast<int32_t>(nt);
+  const int grid = static_cast<int>(std::min<int64_t>(nt, di.sms));
+  return a.M <= 1 ? launch_rows_mt<1>(prm, grid, st, di) : launch_rows_mt<2>(prm, grid, st, di);
+}
+
 struct HPlan {
   int mt;
   int tv;
@@ -334,6 +537,7 @@ namespace w4host {
 
 size_t head_workspace_bytes(int64_t M, int64_t K, int64_t V, int sms) {
   if (M <= 0 || K <= 0 || V <= 0) return 0;
+  if (rows_eligible(M, K)) return 0;
   const HPlan pl = head_plan(M, K, V, sms);
   return COUNTER_BYTES + static_cast<size_t>(pl.grid) * 2 * pl.mt * pl.tv * sizeof(float);
 }
@@ -341,6 +545,7 @@ size_t head_workspace_bytes(int64_t M, int64_t K, int64_t V, int sms) {
 w4_status launch_head(const HeadArgs& a, void* ws, size_t ws_size, cudaStream_t st, const DeviceInfo& di) {
   if (a.K > 0x7fffffff || a.V > 0x7fffffff || a.M > 0x7fffffff)
     return fail(W4_ERR_SHAPE, "head sizes must be below 2^31 on the fast path");
+  if (rows_eligible(a.M, a.K)) return launch_rows(a, st, di);
   const HPlan pl = head_plan(a.M, a.K, a.V, di.sms);
   const size_t need = head_workspace_bytes(a.M, a.K, a.V, di.sms);
   if (ws == nullptr || ws_size < need)
