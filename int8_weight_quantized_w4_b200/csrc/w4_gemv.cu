@@ -13,18 +13,17 @@
 //    32 rows (one K-block) of a narrow one. All matrices of a launch form one
 //    flat range of units; CTA i (one per SM, persistent) takes
 //    [i*W/G, (i+1)*W/G), so every SM streams the same bytes (stream-K).
-//  * A tile whose K-range straddles CTAs is finished by the CTA holding its
-//    largest piece (one whose whole range lies inside the tile, if there is
-//    one; else the larger end piece), so every other piece is at most half a
-//    tile. Every other
+//  * A tile whose K-range straddles CTAs is finished by one of them, chosen on
+//    the host (a CTA whose whole range lies inside the tile, if any; else one
+//    of the two, so that no CTA publishes more than about half of its range).
+//    Every other
 //    contributor writes its partial sums to one of its two workspace slots and
 //    bumps a counter (indexed by the tile's first CTA); the finisher waits
 //    (bounded) until the count is complete, adds the others' partials in CTA
 //    order to its own and resets the counter to zero. The launch is
 //    cooperative, so all CTAs are resident and the finisher's wait ends.
 //  * A CTA walks its range as segments (one tile each): the pieces it
-//    publishes first (at most two, each at most half a tile), then its whole
-//    tiles, then the pieces it finishes. Partials are therefore published
+//    publishes first, then its whole tiles, then the pieces it finishes. Partials are therefore published
 //    early, and the finisher's epilogue warp
 //    collects them before it needs them: a round trip to global memory while
 //    every SM streams takes microseconds, and none is left on the finisher's
@@ -58,6 +57,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <vector>
 
 #include "w4_device.cuh"
 #include "w4_internal.h"
@@ -109,6 +109,10 @@ struct MatParams {
 struct GemvParams {
   MatParams mat[W4_GROUP_MAX];
   uint8_t cta_g[GRID_MAX][2];  // first and last matrix that each CTA's range touches
+  // Split-tile roles of each CTA: bit 0 set when it finishes the tile holding
+  // its first unit, bit 1 the tile holding its last unit (only meaningful
+  // when that tile straddles CTAs). Chosen on the host, see cta_roles().
+  uint8_t cta_fin[GRID_MAX];
   int64_t W;  // total units
   float* ws_partials;
   int32_t* ws_counters;
@@ -185,20 +189,6 @@ __device__ __forceinline__ int64_t cta_of(int64_t f, int64_t W, int64_t G) { ret
 
 __device__ __forceinline__ int64_t range_lo(int64_t i, int64_t W, int64_t G) { return (i * W) / G; }
 
-// The CTA that finishes a split tile [t_start, t_start + t_units): the one
-// holding its largest piece. With a CTA whose whole range lies inside the tile
-// that is this CTA (the last such); otherwise the larger of the two end
-// pieces, the first CTA on a tie. Every other piece is at most half a tile.
-__device__ __forceinline__ int64_t finisher_of(int64_t t_start, int64_t t_units, int64_t W, int64_t G) {
-  const int64_t t_end = t_start + t_units;
-  const int64_t c_first = cta_of(t_start, W, G);
-  const int64_t c_last = cta_of(t_end - 1, W, G);
-  if (c_last - c_first >= 2) return c_last - 1;
-  const int64_t a = range_lo(c_first + 1, W, G) - t_start;  // piece of c_first
-  const int64_t b = t_end - range_lo(c_last, W, G);         // piece of c_last
-  return a >= b ? c_first : c_last;
-}
-
 // The segments of a CTA's range [lo, hi), in processing order. The piece at
 // the start (up to the end of the tile holding lo) and the piece at the end
 // (from the start of the tile holding hi-1) each go first when this CTA
@@ -216,7 +206,7 @@ struct SegIter {
 };
 
 __device__ __noinline__ void seg_init(SegIter& it, const MatScalars* ms, int g0, int g1, int64_t lo, int64_t hi,
-                                      int64_t W, int64_t G) {
+                                      int fin) {
   it.lo = lo;
   it.hi = hi;
   it.k = 0;
@@ -229,12 +219,11 @@ __device__ __noinline__ void seg_init(SegIter& it, const MatScalars* ms, int g0,
   if (it.hd_end == hi) {
     it.tl_start = hi;
   } else {
-    const int64_t me = blockIdx.x;
-    if (a.unit > 0) it.head_late = finisher_of(lo - a.unit, a.tile_units, W, G) == me;
+    if (a.unit > 0) it.head_late = (fin & 1) != 0;
     const Pos b = locate(ms, g1, hi - 1, a.g);
     it.tl_start = hi - 1 - b.unit;
     // a last piece that is a whole tile waits for nobody: it may as well go last
-    it.tail_late = it.tl_start + b.tile_units == hi || finisher_of(it.tl_start, b.tile_units, W, G) == me;
+    it.tail_late = it.tl_start + b.tile_units == hi || (fin & 2) != 0;
   }
   it.f = it.hd_end;
 }
@@ -446,7 +435,9 @@ struct SegInfo {
   int64_t c_first, c_last;
 };
 
-__device__ __noinline__ SegInfo seg_info(const MatScalars* ms, const Pos& ps, int64_t a, int64_t W, int64_t G) {
+// a: first unit of the segment; lo: first unit of this CTA's range; fin: its role bits.
+__device__ __noinline__ SegInfo seg_info(const MatScalars* ms, const Pos& ps, int64_t a, int64_t lo, int fin,
+                                         int64_t W, int64_t G) {
   SegInfo s;
   s.m = &ms[ps.g];
   s.col0 = ps.col0;
@@ -457,7 +448,7 @@ __device__ __noinline__ SegInfo seg_info(const MatScalars* ms, const Pos& ps, in
   s.c_first = cta_of(t_start, W, G);
   s.c_last = cta_of(t_start + ps.tile_units - 1, W, G);
   s.split = s.c_first != s.c_last;
-  s.owner = s.split && static_cast<int64_t>(blockIdx.x) == finisher_of(t_start, ps.tile_units, W, G);
+  s.owner = s.split && (fin & (a == lo ? 1 : 2)) != 0;
   return s;
 }
 
@@ -656,7 +647,7 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
     int it = 0;
     bool ok = true;
     SegIter si;
-    seg_init(si, ms, g0, g1, lo, hi, p.W, G);
+    seg_init(si, ms, g0, g1, lo, hi, p.cta_fin[blockIdx.x]);
     int64_t sa, sb;
     while (ok && seg_next(si, ms, sa, sb)) {
       const Pos ps = locate(ms, g1, sa, g0);
@@ -731,14 +722,14 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
       const int e = warp - 1 - C::NCW;  // takes segments k with k % 2 == e, in buffer e
       const float* rb = red + e * C::RED_FLOATS;
       SegIter si;
-      seg_init(si, ms, g0, g1, lo, hi, p.W, G);
+      seg_init(si, ms, g0, g1, lo, hi, p.cta_fin[blockIdx.x]);
       int64_t sa, sb;
       int k = 0;
       while (seg_next(si, ms, sa, sb)) {
         if ((k & 1) == e) {
           const uint32_t use = static_cast<uint32_t>(k >> 1);
           const Pos ps = locate(ms, g1, sa, g0);
-          const SegInfo info = seg_info(ms, ps, sa, p.W, G);
+          const SegInfo info = seg_info(ms, ps, sa, lo, p.cta_fin[blockIdx.x], p.W, G);
           const auto wsync = [] { __syncwarp(); };
           const auto wbcast = [](int v) { return __shfl_sync(0xffffffffu, v, 0); };
           float* S = own + e * MT * WIDE_N;
@@ -768,7 +759,7 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
   int it = 0;
   bool ok = true;
   SegIter si;
-  seg_init(si, ms, g0, g1, lo, hi, p.W, G);
+  seg_init(si, ms, g0, g1, lo, hi, p.cta_fin[blockIdx.x]);
   int64_t sa, sb;
   int k = 0;
   while (seg_next(si, ms, sa, sb)) {
@@ -833,7 +824,7 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
       if (lane == 0) mbar_arrive(&red_full[rbi]);
     } else {
       named_bar_sync(1, C::NCW * 32);
-      const SegInfo info = seg_info(ms, ps, sa, p.W, G);
+      const SegInfo info = seg_info(ms, ps, sa, lo, p.cta_fin[blockIdx.x], p.W, G);
       const auto bsync = [] { named_bar_sync(1, C::NCW * 32); };
       const auto bbcast = [bcast_slot, ctid](int v) {
         if (ctid == 0) *bcast_slot = v;
@@ -900,6 +891,125 @@ void tiling(int64_t N, int64_t nb, int64_t rmin, int32_t* ntw, int32_t* nnar) {
   else if (rem > 0) nar = 1;
   *ntw = static_cast<int32_t>(w);
   *nnar = nar;
+}
+
+// Split-tile roles of CTAs whose ranges are [c*W/G, (c+1)*W/G): bit 0 of
+// fin[c] set when c finishes the tile holding its first unit (also the one
+// bit read when its whole range lies in one tile), bit 1 when it finishes the
+// tile holding its last unit. Each tile that straddles CTAs gets exactly one
+// finisher; the other contributors publish their pieces, which they process
+// first (the piece at the start of the range, then the one at its end), so a
+// published piece is done after the units its CTA publishes up to and
+// including it. The finisher processes its piece last, so a publish done
+// late in its CTA's range can make the finisher wait; the assignment
+// minimises the sum over published pieces of late(f) = max(0, f - 1/2)^2, f
+// the completion as a fraction of the CTA's range (dynamic programming over
+// the CTAs, the state being whether a CTA publishes the piece at its start). A tile that holds
+// some CTA's whole range is finished by the last such CTA: a range inside one
+// tile cannot be published early.
+// tile_of(f, &start, &units) gives the tile holding flat unit f.
+template <class TileOf>
+void cta_roles(int64_t W, int G, TileOf tile_of, uint8_t* fin) {
+  auto rlo = [&](int64_t c) { return c * W / G; };
+  auto cta = [&](int64_t f) { return ((f + 1) * G + W - 1) / W - 1; };
+  constexpr double kInf = 1e30;
+  auto late = [](double f) { return f > 0.5 ? (f - 0.5) * (f - 0.5) : 0.0; };
+  for (int c = 0; c < G; ++c) fin[c] = 0;
+  // dp[c][s]: least cost of the decisions left of CTA c, with s = 1
+  // when c publishes the piece at the start of its range (of size head[c])
+  std::vector<double> dp0(G + 1, kInf), dp1(G + 1, kInf);
+  std::vector<int64_t> head(G + 1, 0);
+  // how each CTA's state was reached: kind 0 none, 1 forced span from `from`,
+  // 2 c-1 published (A), 3 c published its start (B); prev = state of c-1 / from
+  std::vector<int> kind0(G + 1, 0), kind1(G + 1, 0), prev0(G + 1, 0), prev1(G + 1, 0), from0(G + 1, 0),
+      from1(G + 1, 0);
+  dp0[0] = 0.0;
+  int c = 0;
+  while (c + 1 < G) {
+    const int64_t lo = rlo(c), hi = rlo(c + 1);
+    int64_t ts, tu;
+    tile_of(hi - 1, &ts, &tu);
+    const int64_t te = ts + tu;
+    const double best_any = std::min(dp0[c], dp1[c]);
+    const int arg_any = dp1[c] < dp0[c] ? 1 : 0;
+    if (te <= hi) {  // the range ends at a tile end
+      if (best_any < dp0[c + 1]) {
+        dp0[c + 1] = best_any;
+        kind0[c + 1] = 0;
+        prev0[c + 1] = arg_any;
+      }
+      ++c;
+      continue;
+    }
+    const int cl = static_cast<int>(cta(te - 1));
+    const double R = static_cast<double>(hi - lo);
+    const int64_t a = hi - ts;  // c's piece (the end of its range)
+    if (cl - c >= 2) {
+      // forced: c and cl publish, the last CTA inside finishes, any other CTA
+      // inside publishes its whole range
+      const int64_t b = te - rlo(cl);
+      double span = late(static_cast<double>(b) / static_cast<double>(rlo(cl + 1) - rlo(cl)));
+      if (cl - c >= 3) span += late(1.0) * (cl - c - 2);
+      for (int st = 0; st < 2; ++st) {
+        const double base = st ? dp1[c] : dp0[c];
+        if (base >= kInf) continue;
+        const double v = base + late(static_cast<double>((st ? head[c] : 0) + a) / R) + span;
+        if (v < dp1[cl]) {
+          dp1[cl] = v;
+          kind1[cl] = 1;
+          prev1[cl] = st;
+          from1[cl] = c;
+        }
+      }
+      head[cl] = b;
+      c = cl;
+      continue;
+    }
+    const int64_t b = te - hi;  // c+1's piece (the start of its range)
+    const double R1 = static_cast<double>(rlo(c + 2) - hi);
+    head[c + 1] = b;
+    for (int st = 0; st < 2; ++st) {
+      const double base = st ? dp1[c] : dp0[c];
+      if (base >= kInf) continue;
+      // A: c publishes its piece, c+1 finishes
+      const double va = base + late(static_cast<double>((st ? head[c] : 0) + a) / R);
+      if (va < dp0[c + 1]) {
+        dp0[c + 1] = va;
+        kind0[c + 1] = 2;
+        prev0[c + 1] = st;
+      }
+    }
+    // B: c finishes, c+1 publishes its first piece
+    const double vb = best_any + late(static_cast<double>(b) / R1);
+    if (vb < dp1[c + 1]) {
+      dp1[c + 1] = vb;
+      kind1[c + 1] = 3;
+      prev1[c + 1] = arg_any;
+    }
+    ++c;
+  }
+  // walk back from the better final state, setting the finishers
+  int st = dp1[G - 1] < dp0[G - 1] ? 1 : 0;
+  c = G - 1;
+  while (c > 0) {
+    const int kind = st ? kind1[c] : kind0[c];
+    const int pv = st ? prev1[c] : prev0[c];
+    if (kind == 1) {  // forced span from `from` to c
+      const int f = st ? from1[c] : from0[c];
+      fin[c - 1] |= 3;
+      c = f;
+      st = pv;
+      continue;
+    }
+    const int64_t hi = rlo(c);  // boundary between c-1 and c
+    int64_t ts, tu;
+    tile_of(hi - 1, &ts, &tu);
+    const int64_t te = ts + tu;
+    if (kind == 2) fin[c] |= (rlo(c + 1) <= te) ? 3 : 1;   // c finishes its first piece (or whole range)
+    if (kind == 3) fin[c - 1] |= (ts == rlo(c - 1)) ? 3 : 2;  // c-1 finishes its last piece (or whole range)
+    c -= 1;
+    st = pv;
+  }
 }
 
 struct Plan {
@@ -996,6 +1106,23 @@ w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cud
   }
   if (uoff != pl.W) return fail(W4_ERR_SHAPE, "internal: tiling covers %lld units, plan %lld", static_cast<long long>(uoff),
                                 static_cast<long long>(pl.W));
+  {
+    const int ng = g;
+    auto tile_of = [&](int64_t f, int64_t* start, int64_t* units) {
+      int gi = 0;
+      while (gi + 1 < ng && prm.mat[gi + 1].s.u_off <= f) ++gi;
+      const MatScalars& m = prm.mat[gi].s;
+      const int64_t local = f - m.u_off;
+      if (local < m.u_wide) {
+        *units = 2 * m.nb;
+        *start = f - local % *units;
+      } else {
+        *units = m.nb;
+        *start = f - (local - m.u_wide) % *units;
+      }
+    };
+    cta_roles(uoff, pl.grid, tile_of, prm.cta_fin);
+  }
   prm.count = g;
   prm.W = uoff;
   // first and last matrix of each CTA's range [c*W/G, (c+1)*W/G)
