@@ -49,6 +49,27 @@ def head_bytes() -> int:
     return synth.i8_head_bytes(HEAD_K, HEAD_V)
 
 
+def profiled_traffic(summary: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    recorded in an ncu summary under profiles/, or None when the kernel's
+    source has changed since that capture (its hash no longer matches)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", summary)
+    try:
+        fields = {}
+        for line in open(path):
+            if ":" in line and line.startswith("    "):
+                k, v = line.strip().split(":", 1)
+                fields[k.strip()] = v.strip()
+        src = os.path.join(ROOT, fields["source"])
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if digest != fields["source_sha256_16"]:
+            return None
+        return int(fields["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -322,7 +343,9 @@ def run_ours(args, world, rank, local):
         "body_only": {"ms": round(body_avg, 5), "GB_per_s": round(achieved, 1),
                       "tokens_per_s": round(1e3 / body_avg, 1)},
         "head_only": {"ms": round(head_avg, 5),
-                      "GB_per_s": round(head_bytes() / (head_avg * 1e-3) / 1e9, 1)},
+                      "GB_per_s": round(head_bytes() / (head_avg * 1e-3) / 1e9, 1),
+                      "frac_of_hbm": round(head_bytes() / (head_avg * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                      "traffic": profiled_traffic("i8_rows_gpt2_head_m1.md")},
         "frac_of_hbm_step": round(value / n / peaks["hbm_gbs"], 4),
         "roofline": {
             "kernel": "w4_gemv_kernel<1> (grouped 48-weight launch)",
@@ -332,7 +355,9 @@ def run_ours(args, world, rank, local):
             "peak_source": f"{peaks['_source']} hbm_gbs (copy, burst)",
             "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": None,
+            "traffic": profiled_traffic("w4_gemv_gpt2_m1.md"),
+            "traffic_source": "profiles/w4_gemv_gpt2_m1.md (ncu dram__bytes_read.sum + dram__bytes_write.sum, "
+                              "one launch; null when the kernel source changed since)",
         },
         "e2e": e2e,
         "gpu_launches": 2 * K,  # in the step graph's timed replay
