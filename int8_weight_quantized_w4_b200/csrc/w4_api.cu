@@ -253,6 +253,8 @@ w4_status w4_unpack_nibbles(const uint8_t* packed, int64_t n, uint8_t* q) {
 size_t w4_matmul_workspace_size(int64_t M, int64_t K, int64_t N) {
   const DeviceInfo* di = nullptr;
   if (current_device(&di) != W4_OK || M <= 0 || K <= 0 || N <= 0 || K % 32 || N % 2) return 0;
+  // the GEMV's need (a call may force the GEMV for any M; the tensor-core and
+  // plain kernels need none)
   w4_desc d = {};
   d.M = M;
   d.K = K;
@@ -270,14 +272,19 @@ static w4_status matmul_one(const w4_desc& d, void* ws, size_t wsb, w4_path path
   if (rc != W4_OK) return rc;
   if (d.K == 0) return launch_zero_fill(d.y, d.ldy, d.M, d.N, st);
   const char* why = "";
+  const char* why_tc = "";
   const bool gemv_ok = gemv_eligible(d, &why);
+  const bool tc_ok = tc_eligible(d, &why_tc);
   switch (path) {
     case W4_PATH_GENERIC: return launch_generic(d, st, *di);
     case W4_PATH_GEMV:
       if (!gemv_ok) return fail(W4_ERR_ALIGN, "%s", why);
       return launch_gemv(&d, 1, ws, wsb, st, *di);
-    case W4_PATH_TC: return fail(W4_ERR_SHAPE, "the tcgen05 path is not available in this build");
+    case W4_PATH_TC:
+      if (!tc_ok) return fail(W4_ERR_ALIGN, "%s", why_tc);
+      return launch_tc(&d, 1, st, *di);
     default:
+      if (d.M > kTcMinM) return tc_ok ? launch_tc(&d, 1, st, *di) : launch_generic(d, st, *di);
       return gemv_ok ? launch_gemv(&d, 1, ws, wsb, st, *di) : launch_generic(d, st, *di);
   }
 }
@@ -299,9 +306,20 @@ size_t w4_matmul_grouped_workspace_size(const w4_desc* descs, int32_t count) {
   const DeviceInfo* di = nullptr;
   if (descs == nullptr || count <= 0 || current_device(&di) != W4_OK) return 0;
   size_t best = 0;
-  for (int32_t i = 0; i < count; i += W4_GROUP_MAX) {
-    const int32_t n = count - i < W4_GROUP_MAX ? count - i : W4_GROUP_MAX;
-    const size_t b = gemv_workspace_bytes(descs + i, n, di->sms);
+  // the GEMV takes the descriptors with M <= kTcMinM, W4_GROUP_MAX per launch
+  static thread_local w4_desc small[W4_GROUP_MAX];
+  int n = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    if (descs[i].M > kTcMinM) continue;
+    small[n++] = descs[i];
+    if (n == W4_GROUP_MAX || i == count - 1) {
+      const size_t b = gemv_workspace_bytes(small, n, di->sms);
+      best = b > best ? b : best;
+      n = 0;
+    }
+  }
+  if (n > 0) {
+    const size_t b = gemv_workspace_bytes(small, n, di->sms);
     best = b > best ? b : best;
   }
   return best;
@@ -324,16 +342,28 @@ w4_status w4_matmul_grouped(const w4_desc* descs, int32_t count, void* workspace
   w4_status rc = current_device(&di);
   if (rc != W4_OK) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // Split: descriptors the GEMV can take go into grouped launches; the rest
-  // (K = 0, odd layouts) run one by one on their own kernels.
+  // Split: descriptors with M <= kTcMinM that the GEMV can take go into
+  // grouped GEMV launches, larger M into grouped tensor-core launches; the
+  // rest (K = 0, odd layouts) run one by one on their own kernels.
   static thread_local w4_desc fast[W4_GROUP_MAX];
-  int nfast = 0;
+  static thread_local w4_desc tc[W4_GROUP_MAX];
+  int nfast = 0, ntc = 0;
   for (int32_t i = 0; i < count; ++i) {
     const w4_desc& d = descs[i];
     if (d.M == 0 || d.N == 0) continue;
     const char* why = "";
     if (d.K == 0) {
       rc = launch_zero_fill(d.y, d.ldy, d.M, d.N, st);
+    } else if (d.M > kTcMinM) {
+      if (!tc_eligible(d, &why)) {
+        rc = launch_generic(d, st, *di);
+      } else {
+        tc[ntc++] = d;
+        if (ntc == W4_GROUP_MAX) {
+          rc = launch_tc(tc, ntc, st, *di);
+          ntc = 0;
+        }
+      }
     } else if (!gemv_eligible(d, &why)) {
       rc = launch_generic(d, st, *di);
     } else {
@@ -346,6 +376,8 @@ w4_status w4_matmul_grouped(const w4_desc* descs, int32_t count, void* workspace
     if (rc != W4_OK) return rc;
   }
   if (nfast > 0) rc = launch_gemv(fast, nfast, workspace, workspace_bytes, st, *di);
+  if (rc != W4_OK) return rc;
+  if (ntc > 0) rc = launch_tc(tc, ntc, st, *di);
   return rc;
 }
 

@@ -45,6 +45,10 @@ size_t gemv_workspace_bytes(const w4_desc* d, int count, int sms);
 w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cudaStream_t st,
                       const DeviceInfo& di);
 w4_status launch_generic(const w4_desc& d, cudaStream_t st, const DeviceInfo& di);
+// tcgen05 3xTF32 tile GEMM for M above kTcMinM (no workspace)
+constexpr int64_t kTcMinM = 16;
+bool tc_eligible(const w4_desc& d, const char** why);
+w4_status launch_tc(const w4_desc* d, int count, cudaStream_t st, const DeviceInfo& di);
 w4_status launch_zero_fill(float* y, int64_t ldy, int64_t M, int64_t N, cudaStream_t st);
 
 // ---- head kernels
