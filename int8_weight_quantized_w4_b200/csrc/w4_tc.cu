@@ -3,20 +3,23 @@
 // runtime", section "Quantization (train/quantize.py)", step 2 (dq4): blocks
 // of 32 along K, fp32 scale and uint4 zero point per (block, column),
 // w = (q - zp) * scale. The page's output is fp32 compute, so the products are
-// formed as 3xTF32: x = x_hi + x_lo, w = w_hi + w_lo (hi rounded to tf32, lo
-// the exact fp32 remainder, which the tensor core reads to tf32 precision),
-// and D += x_hi w_hi + x_hi w_lo + x_lo w_hi in an fp32 accumulator. The
-// dropped x_lo w_lo term and the tf32 reading of the lo parts are below
-// 2^-21 |x w| per product.
+// formed as 3xTF32: x = x_hi + x_lo, w = w_hi + w_lo (hi truncated to tf32,
+// lo the exact fp32 remainder, which the tensor core reads to tf32
+// precision), and D += x_hi w_hi + x_hi w_lo + x_lo w_hi in an fp32
+// accumulator. The dropped x_lo w_lo term and the tf32 reading of the lo
+// parts are below 2^-19 |x w| per product.
 //
 // Design (sm_100a):
 //  * One CTA per 128 x 256 tile of y (all weights of a grouped launch share
-//    one grid), four warps. The accumulator (128 lanes x 256 fp32 columns)
+//    one grid), eight warps. The accumulator (128 lanes x 256 fp32 columns)
 //    lives in tensor memory, allocated by warp 0.
 //  * Per 32-row K-block (one scale / zero-point row): the threads load x and
-//    the packed weight slice with plain loads, dequantise exactly as the
-//    oracle does ((q - zp) * s, one fp32 rounding), split both into tf32
-//    hi / lo and store them in shared memory in the canonical K-major layout
+//    the packed weight slice with plain loads (the next block's while the
+//    current one is converted), dequantise exactly as the oracle does
+//    ((q - zp) * s, one fp32 rounding, through the exponent trick of
+//    w4_device.cuh), split both into tf32 hi (low 13 mantissa bits cleared)
+//    and lo (the exact remainder), and store them in shared memory in the
+//    canonical K-major layout
 //    without swizzle (core matrices of 8 rows x 16 bytes; the two 16-byte
 //    halves of an 8-wide K step are LBO = 128 bytes apart, groups of 8 rows
 //    SBO = 256 bytes apart). Two stages: the next block is converted while
@@ -24,8 +27,12 @@
 //  * One thread issues the 12 MMAs of a block (4 K steps x 3 products,
 //    M = 128, N = 256, K = 8, kind::tf32) and commits them to the stage's
 //    mbarrier; the stage is rewritten only after that commit arrives.
-//  * Epilogue: each warp reads its 32 TMEM lanes (rows) 32 columns at a time
-//    and writes y.
+//  * Column 8 l + c of a tile (l = 0..31, c = 0..7) is stored as row 32 c + l
+//    of the B operand, so that the 32 lanes of a warp, which convert the
+//    8-column groups l = 0..31, store contiguous runs (no bank conflicts);
+//    accumulator column j therefore holds y column 8 (j mod 32) + j / 32.
+//  * Epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (its rows) and
+//    columns 128 (w / 4) .. +127, 32 at a time, and writes y.
 // Every wait is bounded; on timeout the kernel records an error and skips
 // the remaining work.
 #include <cuda_runtime.h>
@@ -42,7 +49,7 @@ using namespace w4dev;
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 32;
-constexpr int NT = 128;                                 // 4 warps, one per TMEM lane quadrant
+constexpr int NT = 256;                                 // 8 warps; warp w reads TMEM lanes 32 (w % 4) ..
 constexpr int A_PART = BM * BK * 4;                     // 16 KB: x hi or x lo
 constexpr int B_PART = BN * BK * 4;                     // 32 KB: w hi or w lo
 constexpr int STAGE_BYTES = 2 * A_PART + 2 * B_PART;    // 96 KB
@@ -110,11 +117,9 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__device__ __forceinline__ float tf32_hi(float v) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(v));
-  return __uint_as_float(r);
-}
+// High part of the 3xTF32 split: v with its low 13 mantissa bits cleared (a
+// tf32 value); v - hi is then exact in fp32.
+__device__ __forceinline__ float tf32_hi(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
@@ -165,8 +170,46 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
 
   bool ok = true;
   int issued = 0;  // K-blocks whose MMAs were issued
+  // One K-block's raw inputs for this thread: 4 x (16 bytes of x) and one
+  // 8-column x 4-row piece of the weight with its scales and zero points.
+  // The next block's are loaded while the current one is converted.
+  struct Raw {
+    float4 xv[(BM * BK / 4) / NT];
+    uint32_t w[4];
+    float4 s0, s1;
+    uint32_t z;
+  };
+  const int cg = tid & 31;  // weight: group of 8 columns
+  const int kq = tid >> 5;  // weight: group of 4 rows of the K-block
+  const int nw = n0 + 8 * cg;
+  auto load = [&](int b, Raw& R) {
+    const int k0 = b * BK;
+#pragma unroll
+    for (int i = 0; i < (BM * BK / 4) / NT; ++i) {
+      const int r = tid & (BM - 1), q = (tid >> 7) + 2 * i;
+      const int row = m0 + r;
+      R.xv[i] = row < m.M ? __ldg(reinterpret_cast<const float4*>(m.x + static_cast<int64_t>(row) * m.ldx + k0 + 4 * q))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (nw < m.N) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        R.w[t] = __ldg(reinterpret_cast<const uint32_t*>(m.qw + static_cast<int64_t>(k0 + 4 * kq + t) * hrow + nw / 2));
+      R.s0 = __ldg(reinterpret_cast<const float4*>(m.scales + static_cast<int64_t>(b) * m.N + nw));
+      R.s1 = __ldg(reinterpret_cast<const float4*>(m.scales + static_cast<int64_t>(b) * m.N + nw + 4));
+      R.z = __ldg(reinterpret_cast<const uint32_t*>(m.zp + (static_cast<int64_t>(b) * m.N + nw) / 2));
+    } else {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) R.w[t] = 0u;
+      R.s0 = R.s1 = make_float4(0.f, 0.f, 0.f, 0.f);
+      R.z = 0u;
+    }
+  };
+  Raw cur, nxt;
+  if (m.nb > 0) load(0, cur);
   for (int b = 0; b < m.nb; ++b) {
     const int s = b & 1;
+    if (b + 1 < m.nb) load(b + 1, nxt);
     if (b >= NSTAGE && ok)
       ok = mbar_wait_bounded(&mma_done[s], ((b - NSTAGE) >> 1) & 1, p.timeout_ns, abort_flag, p.err, K_TC, 1);
     if (!ok) break;
@@ -175,55 +218,42 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
     uint8_t* a_lo = st + A_PART;
     uint8_t* b_hi = st + 2 * A_PART;
     uint8_t* b_lo = st + 2 * A_PART + B_PART;
-    const int k0 = b * BK;
-
-    // x slice: 128 rows x 32, eight threads per row (16 bytes each)
-#pragma unroll 2
+    // x: 128 rows x 32, 16 bytes per thread and pass; the 32 lanes of a warp
+    // take 32 consecutive rows, so each store is 4 contiguous core-matrix rows
+    // groups (conflict-free)
+#pragma unroll
     for (int i = 0; i < (BM * BK / 4) / NT; ++i) {
-      const int idx = tid + i * NT;
-      const int r = idx >> 3;
-      const int q = idx & 7;
-      const int row = m0 + r;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (row < m.M) v = __ldg(reinterpret_cast<const float4*>(m.x + static_cast<int64_t>(row) * m.ldx + k0 + 4 * q));
+      const int r = tid & (BM - 1), q = (tid >> 7) + 2 * i;
+      const float4 v = cur.xv[i];
       const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
       const float4 l = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
       const uint32_t off = kmaj_off(r, 4 * q, BM);
       *reinterpret_cast<float4*>(a_hi + off) = h;
       *reinterpret_cast<float4*>(a_lo + off) = l;
     }
-    // weight slice: 32 rows x 256 columns; a thread takes 8 columns x 4 rows
-#pragma unroll 1
-    for (int j = 0; j < (BN / 8) * (BK / 4) / NT; ++j) {
-      const int combo = tid + j * NT;
-      const int cg = combo & 31;  // group of 8 columns
-      const int q = combo >> 5;   // group of 4 rows
-      const int n = n0 + 8 * cg;
-      uint32_t w[4] = {0u, 0u, 0u, 0u};
-      float sv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      uint32_t zw = 0u;
-      if (n < m.N) {
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          w[t] = __ldg(reinterpret_cast<const uint32_t*>(m.qw + static_cast<int64_t>(k0 + 4 * q + t) * hrow + n / 2));
-        const float4 s0 = __ldg(reinterpret_cast<const float4*>(m.scales + static_cast<int64_t>(b) * m.N + n));
-        const float4 s1 = __ldg(reinterpret_cast<const float4*>(m.scales + static_cast<int64_t>(b) * m.N + n + 4));
-        sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
-        sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
-        zw = __ldg(reinterpret_cast<const uint32_t*>(m.zp + (static_cast<int64_t>(b) * m.N + n) / 2));
-      }
+    // weight: w = (q - zp) * s exactly as the oracle rounds it. Nibble c of a
+    // 32-bit word sits at slot c % 4 of its half-word: the float with bits
+    // 0x4B000000 | (half & (0xF << 4 slot)) is 2^23 + q 16^slot exactly, the
+    // difference with the zero point's is (q - zp) 16^slot exactly, and the
+    // scale times 16^-slot (exact) makes the product the oracle's w.
+    {
+      const float sv[8] = {cur.s0.x, cur.s0.y, cur.s0.z, cur.s0.w, cur.s1.x, cur.s1.y, cur.s1.z, cur.s1.w};
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const int zc = static_cast<int>((zw >> (4 * c)) & 15u);
+        const uint32_t zh = c < 4 ? cur.z : cur.z >> 16;
+        const float zf = magic_nib(zh, c & 3);
+        const float sc = sv[c] * inv_slot_scale(c & 3);
         float hv[4], lv[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const int qc = static_cast<int>((w[t] >> (4 * c)) & 15u);
-          const float wv = static_cast<float>(qc - zc) * sv[c];
+          const uint32_t wh = c < 4 ? cur.w[t] : cur.w[t] >> 16;
+          const float wv = (magic_nib(wh, c & 3) - zf) * sc;
           hv[t] = tf32_hi(wv);
           lv[t] = wv - hv[t];
         }
-        const uint32_t off = kmaj_off(8 * cg + c, 4 * q, BN);
+        // column 8 cg + c of the tile is row 32 c + cg of B: a warp's 32
+        // lanes (cg = 0..31) then store 4 contiguous 128-byte runs
+        const uint32_t off = kmaj_off(32 * c + cg, 4 * kq, BN);
         *reinterpret_cast<float4*>(b_hi + off) = make_float4(hv[0], hv[1], hv[2], hv[3]);
         *reinterpret_cast<float4*>(b_lo + off) = make_float4(lv[0], lv[1], lv[2], lv[3]);
       }
@@ -245,6 +275,7 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
       tc_commit(&mma_done[s]);
     }
     issued = b + 1;
+    cur = nxt;
   }
 
   // all MMAs done: the last commit covers every earlier one
@@ -255,17 +286,20 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
   }
   tc_fence_after();
   if (ok && issued == m.nb) {
-    const int row = m0 + 32 * warp + lane;
+    const int quad = warp & 3;  // TMEM lanes 32 quad .. 32 quad + 31 = rows of the tile
+    const int half = warp >> 2; // columns 128 half .. 128 half + 127
+    const int row = m0 + 32 * quad + lane;
 #pragma unroll 1
-    for (int ch = 0; ch < BN / 32; ++ch) {
+    for (int ch = 4 * half; ch < 4 * half + 4; ++ch) {
       uint32_t v[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * ch, v);
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * quad) << 16) + 32 * ch, v);
+      // accumulator column 32 ch + i holds y column 8 i + ch of the tile
       if (row < m.M) {
-        float* yr = m.y + static_cast<int64_t>(row) * m.ldy + n0 + 32 * ch;
-        const int ncol = min(32, m.N - (n0 + 32 * ch));
+        float* yr = m.y + static_cast<int64_t>(row) * m.ldy + n0 + ch;
+        const int ncol = m.N - n0;
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (i < ncol) yr[i] = __uint_as_float(v[i]);
+          if (8 * i + ch < ncol) yr[8 * i] = __uint_as_float(v[i]);
       }
     }
   }
