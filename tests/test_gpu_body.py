@@ -146,7 +146,7 @@ def test_workspace_reused_across_shapes():
     counters must be back at zero after every call."""
     T = torch()
     ws = T.zeros(1 << 22, dtype=T.uint8, device="cuda")
-    for (M, K, N) in [(1, 768, 768), (1, 64, 288), (3, 3072, 768), (1, 64, 288), (8, 96, 544), (1, 8192, 64)]:
+    for (M, K, N) in [(1, 768, 768), (1, 64, 288), (3, 3072, 768), (1, 8224, 64), (8, 96, 544), (1, 8192, 64)]:
         W = synth.w4_weight(K, N, 77)
         x = synth.activations(M, K, 77)
         Wd = upload_w4(W)
@@ -161,8 +161,8 @@ def test_workspace_too_small_is_refused():
     T = torch()
     K, N = 768, 768
     W = upload_w4(synth.w4_weight(K, N))
-    x = dev(synth.activations(1, K))
-    need = w4().w4_matmul_workspace_size(1, K, N)
+    x = dev(synth.activations(2, K))
+    need = w4().w4_matmul_workspace_size(2, K, N)
     assert need > 0
     small = T.zeros(need // 2, dtype=T.uint8, device="cuda")
     with pytest.raises(w4().W4Error) as e:
@@ -180,3 +180,9 @@ def test_bounded_wait_times_out_and_gpu_stays_usable():
     assert w.device_error(clear=False)[0] == 0
     run_case(2, 256, 512, "gemv")  # the context is still healthy
     assert w.device_error(clear=False)[0] == 0
+
+
+def test_m1_long_k():
+    # 257 K-blocks: tall narrow tiles split over several CTAs
+    run_case(1, 8224, 64, "gemv")
+    run_case(1, 8224, 64, "auto")
