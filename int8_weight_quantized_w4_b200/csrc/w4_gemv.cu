@@ -33,7 +33,7 @@
 //    the nibbles (128 rows x 256 B or 256 rows x 128 B), one bulk copy per
 //    K-block of scales and of zero points, and one per row of x, issued by
 //    several lanes at once. A partial stage (at the ends of a segment)
-//    copies unit by unit. Stages form a ring guarded by mbarriers; no copy
+//    copies unit by unit. Stages form a ring of three guarded by mbarriers; no copy
 //    uses multicast. Eight consumer warps dequantise in registers: each takes
 //    16 rows x 256 columns of a stage, a lane owning 8 columns.
 //  * M <= 2: two epilogue warps finish segments (sum over the consumer warps,
@@ -131,7 +131,7 @@ struct Cfg {
   static constexpr int NTHREADS = (1 + NCW + NEPI) * 32;
   static constexpr int X_STAGE = MT * X_ROWS * 4;
   static constexpr int STAGE_BYTES = QW_STAGE + SC_STAGE + ZP_STAGE + X_STAGE;
-  static constexpr int NSTAGES = (MT >= 8) ? 3 : 4;
+  static constexpr int NSTAGES = 3;  // measured best for the GPT-2 body (3 vs 4 stages)
   // per-warp column sums [NCW][MT][256]: handed to the epilogue warps (two
   // buffers, M <= 2) or the accumulators themselves (one buffer, M >= 4)
   static constexpr int RED_FLOATS = NCW * MT * 256;
@@ -323,7 +323,7 @@ template <int MT, bool WIDE, int NCW, int IPW>
 __device__ __forceinline__ void stage_items(const uint8_t* st, int u, int n, int cw, int sub, int lane,
                                             uint32_t kMagic, float2* acc, float* wacc) {
   constexpr int QS = WIDE ? 64 : 32;
-#pragma unroll 1
+#pragma unroll
   for (int ii = 0; ii < IPW; ++ii) {
     const int j = (cw >> 1) + ii * (NCW >> 1);  // unit of the stage for this item
     if (j >= n) continue;

@@ -14,8 +14,8 @@
 //    one grid), eight warps. The accumulator (128 lanes x 256 fp32 columns)
 //    lives in tensor memory, allocated by warp 0.
 //  * Per 32-row K-block (one scale / zero-point row): the threads load x and
-//    the packed weight slice with plain loads (the next block's while the
-//    current one is converted), dequantise exactly as the oracle does
+//    the packed weight slice with plain loads (issued two blocks ahead of
+//    the one being converted), dequantise exactly as the oracle does
 //    ((q - zp) * s, one fp32 rounding, through the exponent trick of
 //    w4_device.cuh), split both into tf32 hi (low 13 mantissa bits cleared)
 //    and lo (the exact remainder), and store them in shared memory in the
@@ -172,7 +172,8 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
   int issued = 0;  // K-blocks whose MMAs were issued
   // One K-block's raw inputs for this thread: 4 x (16 bytes of x) and one
   // 8-column x 4-row piece of the weight with its scales and zero points.
-  // The next block's are loaded while the current one is converted.
+  // The loads of the block after the next are issued while the current one
+  // is converted (two blocks in flight).
   struct Raw {
     float4 xv[(BM * BK / 4) / NT];
     uint32_t w[4];
@@ -205,11 +206,12 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
       R.z = 0u;
     }
   };
-  Raw cur, nxt;
+  Raw cur, nxt, nxt2;
   if (m.nb > 0) load(0, cur);
+  if (m.nb > 1) load(1, nxt);
   for (int b = 0; b < m.nb; ++b) {
     const int s = b & 1;
-    if (b + 1 < m.nb) load(b + 1, nxt);
+    if (b + 2 < m.nb) load(b + 2, nxt2);
     if (b >= NSTAGE && ok)
       ok = mbar_wait_bounded(&mma_done[s], ((b - NSTAGE) >> 1) & 1, p.timeout_ns, abort_flag, p.err, K_TC, 1);
     if (!ok) break;
@@ -276,6 +278,7 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
     }
     issued = b + 1;
     cur = nxt;
+    nxt = nxt2;
   }
 
   // all MMAs done: the last commit covers every earlier one
