@@ -189,6 +189,27 @@ def i8_head_ref(h, table, scales, K: int, V: int, ldt: int | None = None):
     return h64 @ w, np.abs(h64) @ np.abs(w)
 
 
+def i8_embed_ref(table, scales, tokens, K: int, V: int, ldt: int | None = None) -> np.ndarray:
+    """Token lookup from the tied int8 table ("ONNX export, quantization and
+    the browser runtime", section "Quantization (train/quantize.py)", step 3:
+    Gather(axis=1) + Transpose on the [K, V] table, dequantized): row i of the
+    result is column tokens[i] of the table times that token's scale, fp32,
+    one rounding per element. Shape [len(tokens), K]."""
+    ldt = V if ldt is None else ldt
+    if ldt < V:
+        raise ValueError("ldt < V")
+    tok = np.asarray(tokens, dtype=np.int64).reshape(-1)
+    if tok.size and (tok.min() < 0 or tok.max() >= V):
+        raise ValueError("token id out of range")
+    t = np.ascontiguousarray(table, dtype=np.int8).reshape(-1)
+    s = np.ascontiguousarray(scales, dtype=np.float32).reshape(V)
+    out = np.empty((tok.size, K), np.float32)
+    ks = np.arange(K, dtype=np.int64) * ldt
+    for i, v in enumerate(tok):
+        out[i] = t[ks + v].astype(np.float32) * s[v]  # exact int8 -> fp32, one RN multiply
+    return out
+
+
 def last_position_rows(hidden, T: int, K: int) -> np.ndarray:
     """Rows T-1 of M sequences of hidden states [M, T, K] (last_token_logits)."""
     hs = np.asarray(hidden, dtype=np.float32).reshape(-1, T, K)

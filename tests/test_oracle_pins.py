@@ -313,3 +313,43 @@ def test_fp32_blocked_sum_meets_tolerance():
     part = (x.reshape(K // 32, 32, 1) * w.reshape(K // 32, 32, N)).sum(axis=1, dtype=np.float32)
     y32 = part.sum(axis=0, dtype=np.float32)
     assert oracle.max_violation(y32[None, :], y, a) < 0
+
+
+# ---------------------------------------------------------------- token lookup
+
+def test_embed_literal():
+    """Hand-computed: column t of the [K, V] table times scale t."""
+    table = np.array([[1, -2, 3], [4, 5, -6]], np.int8)  # K = 2, V = 3
+    s = np.array([0.5, 0.25, 2.0], np.float32)
+    e = oracle.i8_embed_ref(table, s, [1, 2, 0], 2, 3)
+    assert np.array_equal(e, np.array([[-0.5, 1.25], [6.0, -12.0], [0.5, 2.0]], np.float32))
+
+
+def test_embed_is_the_head_column():
+    """The head is tied: logit t of h equals h . embed(t) (both in fp64 from
+    the same fp32 weights), for every t."""
+    g = np.random.default_rng(11)
+    K, V = 48, 70
+    table = g.integers(-127, 128, (K, V)).astype(np.int8)
+    s = g.uniform(0.002, 0.01, V).astype(np.float32)
+    h = g.standard_normal((1, K)).astype(np.float32)
+    y, _ = oracle.i8_head_ref(h, table, s, K, V)
+    e = oracle.i8_embed_ref(table, s, np.arange(V), K, V).astype(np.float64)
+    assert np.allclose(e @ h[0].astype(np.float64), y[0], rtol=0, atol=1e-12)
+
+
+def test_embed_padded_rows_and_bounds():
+    g = np.random.default_rng(12)
+    K, V, ldt = 5, 9, 13
+    t = g.integers(-128, 128, (K, V)).astype(np.int8)
+    padded = np.full((K, ldt), 77, np.int8)
+    padded[:, :V] = t
+    s = g.uniform(0.01, 0.1, V).astype(np.float32)
+    toks = [0, 8, 3, 3]
+    assert np.array_equal(oracle.i8_embed_ref(padded.reshape(-1), s, toks, K, V, ldt=ldt),
+                          oracle.i8_embed_ref(t, s, toks, K, V))
+    with pytest.raises(ValueError):
+        oracle.i8_embed_ref(t, s, [9], K, V)
+    with pytest.raises(ValueError):
+        oracle.i8_embed_ref(t, s, [-1], K, V)
+    assert oracle.i8_embed_ref(t, s, [], K, V).shape == (0, K)
