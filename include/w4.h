@@ -109,8 +109,9 @@ typedef struct w4_desc {
  * (0 when none is needed). The workspace starts with a fixed block of
  * 32-bit split-K counters followed by partial sums. It must be device memory,
  * 16-byte aligned,
- * and ZERO-FILLED before its first use; every successful call leaves it
- * zero-filled again, so one zeroing at allocation suffices. Two calls that
+ * and ZERO-FILLED before its first use; every successful call leaves the
+ * counter block zero again (the partial sums need no zeroing), so one
+ * zeroing at allocation suffices. Two calls that
  * may run at the same time must not share a workspace. After a call that
  * reported W4_ERR_TIMEOUT, zero it again before reuse. */
 W4_API size_t w4_matmul_workspace_size(int64_t M, int64_t K, int64_t N);
@@ -167,7 +168,7 @@ W4_API w4_status w4_matmul_grouped(const w4_desc* descs, int32_t count, void* wo
 
 /* Bytes of workspace i8_head_logits needs for this shape on the current
  * device (same rules as w4_matmul's workspace: zero-filled before first use,
- * left zero-filled by every successful call, not shared by calls that may run
+ * counter block left zero by every successful call, not shared by calls that may run
  * at the same time). One workspace of the larger size can serve both ops on
  * one stream. */
 W4_API size_t i8_head_workspace_size(int64_t M, int64_t K, int64_t V);
@@ -187,6 +188,34 @@ W4_API w4_status i8_head_logits_path(const float* h, int64_t ldh, const int8_t* 
                                      const float* scales, float* logits, int64_t ldl, int64_t M,
                                      int64_t K, int64_t V, void* workspace, size_t workspace_bytes,
                                      w4_path path, void* stream);
+
+/* Greedy decoding on the head: tokens[m] = argmax_v logits[m, v] (ties to
+ * the lowest token id), best_logits[m] = that logit when best_logits is not
+ * NULL; the logits are exactly those i8_head_logits computes. The pages
+ * measure greedy decoding ("ONNX export, quantization and the browser
+ * runtime", section "Quantization (train/quantize.py)", measurements: 32
+ * greedy tokens); folding the argmax into the head avoids writing and
+ * re-reading the [M, V] logits. tokens / best_logits: device, M entries.
+ * workspace: i8_head_argmax_workspace_size() bytes, 16-byte aligned, with
+ * the same rules as the other workspaces (zero-filled before first use; every
+ * successful call leaves its leading counter block zero); other rules as
+ * i8_head_logits. */
+W4_API size_t i8_head_argmax_workspace_size(int64_t M, int64_t K, int64_t V);
+W4_API w4_status i8_head_argmax(const float* h, int64_t ldh, const int8_t* table, int64_t ldt,
+                                const float* scales, int64_t M, int64_t K, int64_t V, int32_t* tokens,
+                                float* best_logits, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Token lookup from the tied int8 table: out[i, k] = T[k, tokens[i]] *
+ * s[tokens[i]] (fp32, one rounding per element). "ONNX export, quantization
+ * and the browser runtime", section "Quantization (train/quantize.py)",
+ * step 3: the tied table is stored once, [K, V], and the lookup is
+ * Gather(axis=1) + Transpose on it, dequantized. tokens is a DEVICE int32
+ * array of ntok ids; out is device fp32 [ntok, ldo] with ldo >= K, fully
+ * overwritten. A token id outside [0, V) makes its row zero and records
+ * W4_ERR_VALUE in the device error word (read with w4_device_error). Table
+ * 1-byte aligned (any ldt >= V), scales / out 4-byte aligned. */
+W4_API w4_status i8_embed_lookup(const int8_t* table, int64_t ldt, const float* scales, const int32_t* tokens,
+                                 int64_t ntok, float* out, int64_t ldo, int64_t K, int64_t V, void* stream);
 
 /* ------------------------------------------------------------------ host packing */
 

@@ -172,6 +172,38 @@ def i8_head_logits(h, table, scales, K: int, V: int, ldt: int | None = None, log
     return logits
 
 
+def i8_head_argmax(h, table, scales, K: int, V: int, ldt: int | None = None, stream=None):
+    """Greedy next tokens of the last-position rows h: (tokens int32 [M],
+    best logits fp32 [M]), the argmax of the logits i8_head_logits gives
+    (ties to the lowest token id)."""
+    torch = _torch()
+    M = h.shape[0] if h.dim() == 2 else 1
+    ldt = V if ldt is None else ldt
+    tokens = torch.empty(M, dtype=torch.int32, device=h.device)
+    best = torch.empty(M, dtype=torch.float32, device=h.device)
+    ws = workspace(int(lib().i8_head_argmax_workspace_size(M, K, V)), h.device)
+    st = lib().i8_head_argmax(_ptr(h), _ld(h, K), _ptr(table), ldt, _ptr(scales), M, K, V, _ptr(tokens), _ptr(best),
+                              _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream_handle(stream))
+    _check(st, "i8_head_argmax")
+    return tokens, best
+
+
+def i8_embed_lookup(table, scales, tokens, K: int, V: int, ldt: int | None = None, out=None, stream=None):
+    """out[i, k] = T[k, tokens[i]] * s[tokens[i]]: the token lookup on the tied
+    int8 [K, V] table; tokens is a device int32 tensor."""
+    torch = _torch()
+    ldt = V if ldt is None else ldt
+    n = int(tokens.numel())
+    if tokens.dtype != torch.int32 or not tokens.is_contiguous():
+        raise ValueError("tokens must be a contiguous int32 tensor")
+    if out is None:
+        out = torch.empty((n, K), dtype=torch.float32, device=table.device)
+    st = lib().i8_embed_lookup(_ptr(table), ldt, _ptr(scales), _ptr(tokens), n, _ptr(out), _ld(out, K), K, V,
+                               _stream_handle(stream))
+    _check(st, "i8_embed_lookup")
+    return out
+
+
 # ---------------------------------------------------------------- host packing
 
 def pack_nibbles(q) -> np.ndarray:

@@ -56,6 +56,11 @@ SIGNATURES = {
     "w4_matmul_grouped_workspace_size": (C.c_size_t, [C.POINTER(W4Desc), C.c_int32]),
     "w4_matmul_grouped": (C.c_int, [C.POINTER(W4Desc), C.c_int32, C.c_void_p, C.c_size_t, C.c_void_p]),
     "i8_head_workspace_size": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int64]),
+    "i8_head_argmax_workspace_size": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int64]),
+    "i8_head_argmax": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_int64,
+                                 C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "i8_embed_lookup": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p,
+                                  C.c_int64, C.c_int64, C.c_int64, C.c_void_p]),
     "i8_head_logits": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_int64,
                                  C.c_int64, C.c_int64, C.c_int64, C.c_void_p, C.c_size_t, C.c_void_p]),
     "i8_head_logits_path": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,

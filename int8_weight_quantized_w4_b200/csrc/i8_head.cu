@@ -303,6 +303,50 @@ __global__ void __launch_bounds__(NW * 32, HCfg<MT>::MINB) i8_head_kernel(const 
   }
 }
 
+// ---------------------------------------------------------------- greedy decoding
+
+// A 64-bit key whose unsigned order is the order of (logit, -token): the
+// logit's bits made monotonic (non-negative: sign bit set; negative: all bits
+// flipped) above the complement of the token id, so the maximum key is the
+// largest logit and, among equal logits, the lowest token id. 0 is below
+// every key of a number.
+__device__ __forceinline__ unsigned long long argmax_key(float logit, uint32_t token) {
+  const uint32_t b = __float_as_uint(logit);
+  const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return (static_cast<unsigned long long>(o) << 32) | static_cast<unsigned long long>(0xFFFFFFFFu - token);
+}
+
+__device__ __forceinline__ unsigned long long warp_max_key(unsigned long long k) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) k = max(k, __shfl_xor_sync(0xffffffffu, k, o));
+  return k;
+}
+
+// keys[m] <- max over the logits of row m (for heads whose logits were
+// written to a buffer first).
+__global__ void __launch_bounds__(256) argmax_rows_kernel(const float* __restrict__ logits, int64_t ldl, int32_t V,
+                                                          unsigned long long* keys) {
+  const int m = blockIdx.y;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 2048;
+  unsigned long long best = 0ull;
+  for (int64_t c = c0 + threadIdx.x; c < min(c0 + 2048, static_cast<int64_t>(V)); c += 256)
+    best = max(best, argmax_key(__ldg(logits + m * ldl + c), static_cast<uint32_t>(c)));
+  best = warp_max_key(best);
+  if ((threadIdx.x & 31) == 0 && best != 0ull) atomicMax(keys + m, best);
+}
+
+// tokens[m] (and best[m], when given) from keys[m].
+__global__ void argmax_finish_kernel(const unsigned long long* keys, int32_t M, int32_t* tokens, float* best) {
+  const int m = blockIdx.x * blockDim.x + threadIdx.x;
+  if (m >= M) return;
+  const unsigned long long k = keys[m];
+  tokens[m] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(k & 0xFFFFFFFFull));
+  if (best != nullptr) {
+    const uint32_t o = static_cast<uint32_t>(k >> 32);
+    best[m] = __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+  }
+}
+
 // ---------------------------------------------------------------- i8_rows_kernel
 
 constexpr int RROWS = 64;             // rows per stage
@@ -325,6 +369,9 @@ struct RowsParams {
   int32_t ntiles;  // column slices, [t*V/ntiles, (t+1)*V/ntiles)
   int32_t kpad;    // K rounded up to whole stages
   int32_t pad;
+  // greedy decoding: when set, logits are not written; each CTA folds the
+  // best (logit, token) of its slice into keys[m] (see argmax_key)
+  unsigned long long* keys;
 };
 
 template <int MT>
@@ -436,6 +483,9 @@ __global__ void __launch_bounds__(RTHREADS, 1) i8_rows_kernel(const __grid_const
     if (t < 16)
       shifts[t] = static_cast<int>(reinterpret_cast<uintptr_t>(p.table + static_cast<int64_t>(t) * p.ldt + v0) & 15);
     __syncthreads();
+    unsigned long long best[MT];
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm) best[mm] = 0ull;
     for (int c = t; c < ncols; c += RTHREADS) {
       const float sc = __ldg(p.scales + v0 + c);
 #pragma unroll
@@ -444,7 +494,17 @@ __global__ void __launch_bounds__(RTHREADS, 1) i8_rows_kernel(const __grid_const
         float v = 0.f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) v += red[(mm * 16 + j) * RWIN + c + shifts[j]];
-        p.logits[static_cast<int64_t>(mm) * p.ldl + v0 + c] = v * sc;
+        const float logit = v * sc;
+        if (p.keys == nullptr) p.logits[static_cast<int64_t>(mm) * p.ldl + v0 + c] = logit;
+        else best[mm] = max(best[mm], argmax_key(logit, static_cast<uint32_t>(v0 + c)));
+      }
+    }
+    if (p.keys != nullptr) {
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        if (mm >= p.M) break;
+        const unsigned long long b = warp_max_key(best[mm]);
+        if ((t & 31) == 0 && b != 0ull) atomicMax(p.keys + mm, b);
       }
     }
     __syncthreads();  // red and shifts are reused by the next slice
@@ -472,8 +532,10 @@ bool rows_eligible(int64_t M, int64_t K) {
   return M <= 2 && M * kpad * 4 <= RH_MAX_BYTES;
 }
 
-w4_status launch_rows(const w4host::HeadArgs& a, cudaStream_t st, const w4host::DeviceInfo& di) {
+w4_status launch_rows(const w4host::HeadArgs& a, cudaStream_t st, const w4host::DeviceInfo& di,
+                      unsigned long long* keys = nullptr) {
   RowsParams prm;
+  prm.keys = keys;
   prm.h = a.h;
   prm.ldh = a.ldh;
   prm.table = a.table;
@@ -575,6 +637,28 @@ w4_status launch_head(const HeadArgs& a, void* ws, size_t ws_size, cudaStream_t 
     case 4: return launch_head_mt<4>(prm, pl.grid, st, di);
     default: return launch_head_mt<8>(prm, pl.grid, st, di);
   }
+}
+
+bool head_rows_path(int64_t M, int64_t K) { return K > 0 && rows_eligible(M, K); }
+
+w4_status launch_head_keys(const HeadArgs& a, unsigned long long* keys, cudaStream_t st, const DeviceInfo& di) {
+  return launch_rows(a, st, di, keys);
+}
+
+w4_status launch_argmax_rows(const float* logits, int64_t ldl, int64_t M, int64_t V, unsigned long long* keys,
+                             cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>((V + 2047) / 2048), static_cast<unsigned>(M));
+  argmax_rows_kernel<<<grid, 256, 0, st>>>(logits, ldl, static_cast<int32_t>(V), keys);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W4_OK : cuda_fail(e, "launch argmax_rows");
+}
+
+w4_status launch_argmax_finish(const unsigned long long* keys, int64_t M, int32_t* tokens, float* best,
+                               cudaStream_t st) {
+  argmax_finish_kernel<<<static_cast<unsigned>((M + 127) / 128), 128, 0, st>>>(keys, static_cast<int32_t>(M), tokens,
+                                                                              best);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W4_OK : cuda_fail(e, "launch argmax_finish");
 }
 
 }  // namespace w4host

@@ -407,6 +407,80 @@ static w4_status head_impl(const HeadArgs& a, void* ws, size_t wsb, w4_path path
   return launch_head(a, ws, wsb, st, *di);
 }
 
+// Greedy decoding: when the rows kernel folds the logits itself the workspace
+// is [64-bit keys, M of them]; otherwise [the head's own workspace, so that
+// its counter block sits at the start as always][keys][logits M x V], each
+// part 256-byte aligned.
+static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+static size_t argmax_head_ws(int64_t M, int64_t K, int64_t V, int sms) {
+  return head_rows_path(M, K) ? 0 : round256(head_workspace_bytes(M, K, V, sms));
+}
+
+static size_t argmax_ws_bytes(int64_t M, int64_t K, int64_t V, int sms) {
+  size_t b = argmax_head_ws(M, K, V, sms) + round256(static_cast<size_t>(M) * 8);
+  if (!head_rows_path(M, K)) b += static_cast<size_t>(M) * static_cast<size_t>(V) * 4;
+  return b;
+}
+
+size_t i8_head_argmax_workspace_size(int64_t M, int64_t K, int64_t V) {
+  const DeviceInfo* di = nullptr;
+  if (current_device(&di) != W4_OK || M <= 0 || K < 0 || V <= 0) return 0;
+  return argmax_ws_bytes(M, K, V, di->sms);
+}
+
+w4_status i8_head_argmax(const float* h, int64_t ldh, const int8_t* table, int64_t ldt, const float* scales,
+                         int64_t M, int64_t K, int64_t V, int32_t* tokens, float* best_logits, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (M < 0 || K < 0 || V < 0) return fail(W4_ERR_SHAPE, "negative size");
+  if (M == 0) return W4_OK;
+  if (V == 0) return fail(W4_ERR_SHAPE, "V == 0: no token to choose");
+  if (V > 0x7fffffff || M > 65535) return fail(W4_ERR_SHAPE, "V must be below 2^31 and M at most 65535");
+  if (tokens == nullptr) return fail(W4_ERR_NULL, "tokens is NULL");
+  if (!aligned(tokens, 4) || !aligned(best_logits, 4)) return fail(W4_ERR_ALIGN, "tokens and best must be 4-byte aligned");
+  if (K > 0) {
+    if (h == nullptr || table == nullptr || scales == nullptr)
+      return fail(W4_ERR_NULL, "h, table and scales must not be NULL");
+    if (ldh < K) return fail(W4_ERR_SHAPE, "ldh < K");
+    if (ldt < V) return fail(W4_ERR_SHAPE, "ldt < V");
+    if (!aligned(h, 4) || !aligned(scales, 4)) return fail(W4_ERR_ALIGN, "h and scales must be 4-byte aligned");
+    if (!aligned(table, 16)) return fail(W4_ERR_ALIGN, "table must be 16-byte aligned");
+  }
+  const DeviceInfo* di = nullptr;
+  w4_status rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  const size_t need = argmax_ws_bytes(M, K, V, di->sms);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(W4_ERR_WORKSPACE, "argmax workspace of %zu bytes needed, %zu given", need,
+                workspace == nullptr ? size_t(0) : workspace_bytes);
+  if (!aligned(workspace, 16)) return fail(W4_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t hws_bytes = argmax_head_ws(M, K, V, di->sms);
+  auto* keys = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + hws_bytes);
+  cudaError_t e = cudaMemsetAsync(keys, 0, static_cast<size_t>(M) * 8, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clear argmax keys");
+  if (head_rows_path(M, K)) {
+    const HeadArgs a = {h, ldh, table, ldt, scales, nullptr, V, M, K, V};
+    rc = launch_head_keys(a, keys, st, *di);
+  } else {
+    float* logits = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(keys) + round256(static_cast<size_t>(M) * 8));
+    if (K == 0) {
+      rc = launch_zero_fill(logits, V, M, V, st);
+    } else {
+      const HeadArgs a = {h, ldh, table, ldt, scales, logits, V, M, K, V};
+      rc = launch_head(a, hws_bytes > 0 ? workspace : nullptr, hws_bytes, st, *di);
+    }
+    if (rc == W4_OK) rc = launch_argmax_rows(logits, V, M, V, keys, st);
+  }
+  if (rc != W4_OK) return rc;
+  rc = launch_argmax_finish(keys, M, tokens, best_logits, st);
+  if (rc != W4_OK) return rc;
+  // the keys may lie in the block where other calls keep their counters:
+  // leave them zero, as every call of this library leaves that block
+  e = cudaMemsetAsync(keys, 0, static_cast<size_t>(M) * 8, st);
+  return e == cudaSuccess ? W4_OK : cuda_fail(e, "clear argmax keys");
+}
+
 size_t i8_head_workspace_size(int64_t M, int64_t K, int64_t V) {
   const DeviceInfo* di = nullptr;
   if (current_device(&di) != W4_OK) return 0;

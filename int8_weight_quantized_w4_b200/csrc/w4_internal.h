@@ -65,6 +65,14 @@ struct HeadArgs {
 size_t head_workspace_bytes(int64_t M, int64_t K, int64_t V, int sms);
 w4_status launch_head(const HeadArgs& a, void* ws, size_t ws_size, cudaStream_t st, const DeviceInfo& di);
 w4_status launch_head_generic(const HeadArgs& a, cudaStream_t st, const DeviceInfo& di);
+// greedy decoding: the rows kernel folds its logits into 64-bit keys (M <= 2
+// and h fits its shared memory); otherwise logits are written and reduced
+bool head_rows_path(int64_t M, int64_t K);
+w4_status launch_head_keys(const HeadArgs& a, unsigned long long* keys, cudaStream_t st, const DeviceInfo& di);
+w4_status launch_argmax_rows(const float* logits, int64_t ldl, int64_t M, int64_t V, unsigned long long* keys,
+                             cudaStream_t st);
+w4_status launch_argmax_finish(const unsigned long long* keys, int64_t M, int32_t* tokens, float* best,
+                               cudaStream_t st);
 
 // ---- diagnostics
 w4_status launch_debug_wait(uint64_t timeout_ns, cudaStream_t st, const DeviceInfo& di);

@@ -189,6 +189,21 @@ def i8_head_ref(h, table, scales, K: int, V: int, ldt: int | None = None):
     return h64 @ w, np.abs(h64) @ np.abs(w)
 
 
+def i8_head_argmax_ref(h, table, scales, K: int, V: int, ldt: int | None = None):
+    """Greedy decoding on the head: for each row of h, the token with the
+    largest logit (the lowest id among equal ones), that logit, and the gap
+    to the next-best distinct logit (fp64; inf when V == 1 or all equal)."""
+    y, _ = i8_head_ref(h, table, scales, K, V, ldt)
+    tok = np.argmax(y, axis=1)  # first maximum: the lowest id on ties
+    best = y[np.arange(y.shape[0]), tok]
+    gap = np.full(y.shape[0], np.inf)
+    for m in range(y.shape[0]):
+        rest = y[m][y[m] < best[m]]
+        if rest.size:
+            gap[m] = best[m] - rest.max()
+    return tok.astype(np.int64), best, gap
+
+
 def i8_embed_ref(table, scales, tokens, K: int, V: int, ldt: int | None = None) -> np.ndarray:
     """Token lookup from the tied int8 table ("ONNX export, quantization and
     the browser runtime", section "Quantization (train/quantize.py)", step 3:

@@ -353,3 +353,15 @@ def test_embed_padded_rows_and_bounds():
     with pytest.raises(ValueError):
         oracle.i8_embed_ref(t, s, [-1], K, V)
     assert oracle.i8_embed_ref(t, s, [], K, V).shape == (0, K)
+
+
+# ---------------------------------------------------------------- greedy decoding
+
+def test_argmax_literal_and_ties():
+    """Hand case: h = [1, 2]; columns give logits 0.5*(1+4)=2.5, 0.25*(-2+10)=2,
+    2*(3-12)=-18, 1*(1+4)=5 (twice): the first of the two fives wins."""
+    table = np.array([[1, -2, 3, 1, 1], [2, 5, -6, 2, 2]], np.int8)  # K = 2, V = 5
+    s = np.array([0.5, 0.25, 2.0, 1.0, 1.0], np.float32)
+    h = np.array([[1.0, 2.0]], np.float32)
+    tok, best, gap = oracle.i8_head_argmax_ref(h, table, s, 2, 5)
+    assert tok.tolist() == [3] and best.tolist() == [5.0] and gap.tolist() == [2.5]
