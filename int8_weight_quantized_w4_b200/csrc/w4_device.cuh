@@ -158,10 +158,6 @@ __device__ __forceinline__ void tma_g2s_2d(void* dst, const CUtensorMap* map, in
       : "memory");
 }
 
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
 // ---------------------------------------------------------------- named barriers
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

@@ -166,18 +166,18 @@ __device__ __noinline__ Pos locate(const MatScalars* ms, int g_hi, int64_t f, in
   if (local < m.u_wide) {
     r.wide = true;
     r.tile_units = 2 * m.nb;
-    const int64_t tl = local / r.tile_units;
+    const int64_t tl = static_cast<uint32_t>(local) / static_cast<uint32_t>(r.tile_units);
     r.unit = static_cast<int32_t>(local - tl * r.tile_units);
-    const int32_t tile = static_cast<int32_t>(tl / m.nmc);
+    const int32_t tile = static_cast<int32_t>(static_cast<uint32_t>(tl) / static_cast<uint32_t>(m.nmc));
     r.mc = static_cast<int32_t>(tl - static_cast<int64_t>(tile) * m.nmc);
     r.col0 = tile * WIDE_N;
   } else {
     r.wide = false;
     r.tile_units = m.nb;
     const int64_t l2 = local - m.u_wide;
-    const int64_t tl = l2 / m.nb;
+    const int64_t tl = static_cast<uint32_t>(l2) / static_cast<uint32_t>(m.nb);
     r.unit = static_cast<int32_t>(l2 - tl * m.nb);
-    const int32_t tile = static_cast<int32_t>(tl / m.nmc);
+    const int32_t tile = static_cast<int32_t>(static_cast<uint32_t>(tl) / static_cast<uint32_t>(m.nmc));
     r.mc = static_cast<int32_t>(tl - static_cast<int64_t>(tile) * m.nmc);
     r.col0 = m.ntw * WIDE_N + tile * NARROW_N;
   }
@@ -185,9 +185,16 @@ __device__ __noinline__ Pos locate(const MatScalars* ms, int g_hi, int64_t f, in
 }
 
 // CTA whose range holds flat index f (ranges are [floor(i W / G), floor((i+1) W / G))).
-__device__ __forceinline__ int64_t cta_of(int64_t f, int64_t W, int64_t G) { return ((f + 1) * G + W - 1) / W - 1; }
+// The host guarantees W * G < 2^32, so every product here fits 32 bits and the
+// divisions are 32-bit ones (a 64-bit division is a long subroutine, and these
+// sit on the path to a CTA's first copy).
+__device__ __forceinline__ int64_t cta_of(int64_t f, int64_t W, int64_t G) {
+  return static_cast<uint32_t>((f + 1) * G + W - 1) / static_cast<uint32_t>(W) - 1;
+}
 
-__device__ __forceinline__ int64_t range_lo(int64_t i, int64_t W, int64_t G) { return (i * W) / G; }
+__device__ __forceinline__ int64_t range_lo(int64_t i, int64_t W, int64_t G) {
+  return static_cast<uint32_t>(i * W) / static_cast<uint32_t>(G);
+}
 
 // The segments of a CTA's range [lo, hi), in processing order. The piece at
 // the start (up to the end of the tile holding lo) and the piece at the end
@@ -637,13 +644,6 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 1) w4_gemv_kernel(const __g
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    for (int g = g0 + (lane >> 2); g <= g1; g += 8) {
-      const CUtensorMap* mp = (lane & 3) == 0   ? &p.mat[g].qw_wide_full
-                              : (lane & 3) == 1 ? &p.mat[g].qw_wide_unit
-                              : (lane & 3) == 2 ? &p.mat[g].qw_narrow_full
-                                                : &p.mat[g].qw_narrow_unit;
-      prefetch_tensormap(mp);
-    }
     int it = 0;
     bool ok = true;
     SegIter si;
@@ -1069,6 +1069,10 @@ w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cud
   if (count > W4_GROUP_MAX) return fail(W4_ERR_SHAPE, "at most %d matrices per GEMV launch", W4_GROUP_MAX);
   const Plan pl = make_plan(d, count, di.sms);
   if (pl.W == 0) return W4_OK;
+  // the kernel's flat-index arithmetic is 32-bit: W * grid must stay below 2^32
+  if (pl.W * pl.grid >= (int64_t(1) << 32))
+    return fail(W4_ERR_SHAPE, "%lld units over %d CTAs is beyond one GEMV launch; split the group",
+                static_cast<long long>(pl.W), pl.grid);
   const size_t need = ws_bytes(pl);
   if (ws == nullptr || ws_size < need)
     return fail(W4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws == nullptr ? size_t(0) : ws_size);
