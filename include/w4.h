@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define W4_ABI_VERSION 1
+#define W4_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define W4_API __attribute__((visibility("default")))
@@ -89,7 +89,30 @@ typedef enum w4_path {
   W4_PATH_TC = 3       /* tcgen05 3xTF32 tile GEMM (large M)                                  */
 } w4_path;
 
-/* One independent matmul of a grouped launch; fields as in w4_matmul. */
+/* Activation of the fused epilogue (see w4_desc). GPT-2's MLP uses the
+ * tanh form ("gelu_new"); the erf form is the exact GELU. */
+typedef enum w4_act {
+  W4_ACT_NONE = 0,      /* identity                                                   */
+  W4_ACT_GELU_TANH = 1, /* 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3)))            */
+  W4_ACT_GELU_ERF = 2   /* 0.5 v (1 + erf(v / sqrt(2)))                                */
+} w4_act;
+
+/* One matmul: the fields x .. N as in w4_matmul, then an optional fused
+ * epilogue. The pages' export step "gemm_to_matmul" ("ONNX export,
+ * quantization and the browser runtime", section "Quantization
+ * (train/quantize.py)", step 1) splits every GPT-2 Conv1D into MatMul + Add;
+ * the epilogue folds that Add, and the activation or residual add that
+ * follows it in the model, into the kernel's final store:
+ *   y[m, n] = act(x.W[m, n] + bias[n]) + residual[m * ldr + n]
+ * all in fp32, in that order.
+ * - bias: NULL or [N] fp32, 4-byte aligned.
+ * - residual: NULL or [M, N] fp32 with row stride ldr >= N, 4-byte aligned.
+ *   It may be y itself (same pointer and ldr == ldy: an in-place residual
+ *   update); any other overlap with y or the inputs is not allowed.
+ * - act: a w4_act value; anything else is refused with W4_ERR_VALUE.
+ * - reserved: must be 0.
+ * All-zero epilogue fields (what a zero-initialised struct holds) mean plain
+ * y = x.W. */
 typedef struct w4_desc {
   const float* x;
   int64_t ldx;
@@ -101,6 +124,11 @@ typedef struct w4_desc {
   int64_t M;
   int64_t K;
   int64_t N;
+  const float* bias;
+  const float* residual;
+  int64_t ldr;
+  int32_t act;
+  int32_t reserved;
 } w4_desc;
 
 /* ------------------------------------------------------------------ body */
@@ -123,6 +151,12 @@ W4_API size_t w4_matmul_workspace_size(int64_t M, int64_t K, int64_t N);
 W4_API w4_status w4_matmul(const float* x, int64_t ldx, const uint8_t* qw, const float* scales,
                     const uint8_t* zp, float* y, int64_t ldy, int64_t M, int64_t K, int64_t N,
                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* One matmul described by a w4_desc (epilogue included), with a kernel
+ * choice; the workspace rules are w4_matmul's. `d` is a HOST pointer read
+ * during the call only. */
+W4_API w4_status w4_matmul_desc(const w4_desc* d, void* workspace, size_t workspace_bytes, w4_path path,
+                                void* stream);
 
 /* As w4_matmul with an explicit kernel choice. */
 W4_API w4_status w4_matmul_path(const float* x, int64_t ldx, const uint8_t* qw, const float* scales,

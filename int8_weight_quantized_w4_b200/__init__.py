@@ -7,6 +7,7 @@ nothing falls back to another implementation.
 
 Operations (see include/w4.h for layouts and error behaviour):
   w4_matmul(x, qw, scales, zp, K, N)        y = x . W, W 4-bit blocked
+      (..., bias=, residual=, act=)         y = act(x . W + bias) + residual, fused
   w4_matmul_grouped([...])                  many independent ones, one launch
   i8_head_logits(h, table, scales, K, V)    last-position logits, int8 head
   pack_nibbles / unpack_nibbles             host-side UINT4 packing
@@ -20,7 +21,7 @@ from typing import Sequence
 import numpy as np
 
 from . import _lib
-from ._lib import GROUP_MAX, PATHS, STATUS, W4Desc, W4LibraryMissing  # noqa: F401
+from ._lib import ACTS, GROUP_MAX, PATHS, STATUS, W4Desc, W4LibraryMissing  # noqa: F401
 
 
 class W4Error(RuntimeError):
@@ -101,9 +102,21 @@ def w4_matmul_workspace_size(M: int, K: int, N: int) -> int:
     return int(lib().w4_matmul_workspace_size(M, K, N))
 
 
-def w4_matmul(x, qw, scales, zp, K: int, N: int, y=None, path: str = "auto", ws=None, stream=None):
+def _epilogue(it: dict, N: int):
+    """(bias ptr, residual ptr, ldr, act code) of an item's optional epilogue."""
+    bias, res, act = it.get("bias"), it.get("residual"), it.get("act", "none")
+    if act not in ACTS:
+        raise ValueError(f"act must be one of {sorted(ACTS)}")
+    return _ptr(bias), _ptr(res), (0 if res is None else _ld(res, N)), ACTS[act]
+
+
+def w4_matmul(x, qw, scales, zp, K: int, N: int, y=None, path: str = "auto", ws=None, stream=None, bias=None,
+              residual=None, act: str = "none"):
     """y[M, N] = x[M, K] . W[K, N] (fp32) with W given as packed nibbles,
-    fp32 scales [K/32, N] and packed zero points; returns y."""
+    fp32 scales [K/32, N] and packed zero points; returns y.
+
+    With bias ([N]), residual ([M, N], may be y itself) or act ("gelu_tanh",
+    "gelu_erf") the kernel's final store computes act(x . W + bias) + residual."""
     torch = _torch()
     M = x.shape[0] if x.dim() == 2 else 1
     if y is None:
@@ -111,6 +124,13 @@ def w4_matmul(x, qw, scales, zp, K: int, N: int, y=None, path: str = "auto", ws=
     need = w4_matmul_workspace_size(M, K, N)
     if ws is None:
         ws = workspace(need, x.device)
+    if bias is not None or residual is not None or act != "none":
+        b, r, ldr, a = _epilogue({"bias": bias, "residual": residual, "act": act}, N)
+        d = W4Desc(_ptr(x), _ld(x, K), _ptr(qw), _ptr(scales), _ptr(zp), _ptr(y), _ld(y, N), M, K, N, b, r, ldr, a, 0)
+        st = lib().w4_matmul_desc(C.byref(d), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                  PATHS[path], _stream_handle(stream))
+        _check(st, "w4_matmul")
+        return y
     st = lib().w4_matmul_path(_ptr(x), _ld(x, K), _ptr(qw), _ptr(scales), _ptr(zp), _ptr(y), _ld(y, N), M, K, N,
                               _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), PATHS[path],
                               _stream_handle(stream))
@@ -120,14 +140,16 @@ def w4_matmul(x, qw, scales, zp, K: int, N: int, y=None, path: str = "auto", ws=
 
 def make_descs(items: Sequence[dict]):
     """ctypes descriptor array for w4_matmul_grouped; each item holds the
-    tensors x, qw, scales, zp, y and the ints K, N (M from x)."""
+    tensors x, qw, scales, zp, y and the ints K, N (M from x), and optionally
+    the fused epilogue "bias", "residual" and "act" (as in w4_matmul)."""
     arr = (W4Desc * len(items))()
     for i, it in enumerate(items):
         x, y = it["x"], it["y"]
         K, N = int(it["K"]), int(it["N"])
         M = x.shape[0] if x.dim() == 2 else 1
+        b, r, ldr, a = _epilogue(it, N)
         arr[i] = W4Desc(_ptr(x), _ld(x, K), _ptr(it["qw"]), _ptr(it["scales"]), _ptr(it["zp"]), _ptr(y),
-                        _ld(y, N), M, K, N)
+                        _ld(y, N), M, K, N, b, r, ldr, a, 0)
     return arr
 
 

@@ -26,6 +26,8 @@ STATUS = {
 W4_OK, W4_ERR_NULL, W4_ERR_SHAPE, W4_ERR_ALIGN, W4_ERR_DEVICE, W4_ERR_CUDA, W4_ERR_TIMEOUT, W4_ERR_WORKSPACE, \
     W4_ERR_VALUE = range(9)
 PATHS = {"auto": 0, "gemv": 1, "generic": 2, "tc": 3}
+ACTS = {"none": 0, "gelu_tanh": 1, "gelu_erf": 2}
+ABI_VERSION = 2
 GROUP_MAX = 48
 
 
@@ -41,6 +43,11 @@ class W4Desc(C.Structure):
         ("M", C.c_int64),
         ("K", C.c_int64),
         ("N", C.c_int64),
+        ("bias", C.c_void_p),
+        ("residual", C.c_void_p),
+        ("ldr", C.c_int64),
+        ("act", C.c_int32),
+        ("reserved", C.c_int32),
     ]
 
 
@@ -53,6 +60,7 @@ SIGNATURES = {
                                  C.c_int64, C.c_int64, C.c_int64, C.c_void_p, C.c_size_t, C.c_int, C.c_void_p]),
     "w4_matmul_noalloc": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                     C.c_int64, C.c_int64, C.c_int64, C.c_int64, C.c_void_p]),
+    "w4_matmul_desc": (C.c_int, [C.POINTER(W4Desc), C.c_void_p, C.c_size_t, C.c_int, C.c_void_p]),
     "w4_matmul_grouped_workspace_size": (C.c_size_t, [C.POINTER(W4Desc), C.c_int32]),
     "w4_matmul_grouped": (C.c_int, [C.POINTER(W4Desc), C.c_int32, C.c_void_p, C.c_size_t, C.c_void_p]),
     "i8_head_workspace_size": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int64]),
@@ -97,5 +105,8 @@ def load():
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
+    if lib.w4_abi_version() != ABI_VERSION:
+        raise W4LibraryMissing(f"{LIB_PATH} has ABI version {lib.w4_abi_version()}, this binding needs "
+                               f"{ABI_VERSION}: rebuild it")
     _lib = lib
     return lib

@@ -182,10 +182,19 @@ static w4_status check_desc(const w4_desc& d) {
                                                  (long long)d.M, (long long)d.K, (long long)d.N);
   if (d.K % 32 != 0) return fail(W4_ERR_SHAPE, "K=%lld is not a multiple of 32", (long long)d.K);
   if (d.N % 2 != 0) return fail(W4_ERR_SHAPE, "N=%lld is odd", (long long)d.N);
+  if (d.act < W4_ACT_NONE || d.act > W4_ACT_GELU_ERF) return fail(W4_ERR_VALUE, "unknown activation %d", int(d.act));
+  if (d.reserved != 0) return fail(W4_ERR_VALUE, "reserved field must be 0");
   if (d.M == 0 || d.N == 0) return W4_OK;
   if (d.y == nullptr) return fail(W4_ERR_NULL, "y is NULL");
   if (d.ldy < d.N) return fail(W4_ERR_SHAPE, "ldy=%lld < N=%lld", (long long)d.ldy, (long long)d.N);
   if (!aligned(d.y, 4)) return fail(W4_ERR_ALIGN, "y must be 4-byte aligned");
+  if (d.bias != nullptr && !aligned(d.bias, 4)) return fail(W4_ERR_ALIGN, "bias must be 4-byte aligned");
+  if (d.residual != nullptr) {
+    if (d.ldr < d.N) return fail(W4_ERR_SHAPE, "ldr=%lld < N=%lld", (long long)d.ldr, (long long)d.N);
+    if (!aligned(d.residual, 4)) return fail(W4_ERR_ALIGN, "residual must be 4-byte aligned");
+    if (d.residual == d.y && d.ldr != d.ldy)
+      return fail(W4_ERR_SHAPE, "an in-place residual (residual == y) needs ldr == ldy");
+  }
   if (d.K == 0) return W4_OK;
   if (d.x == nullptr || d.qw == nullptr || d.scales == nullptr || d.zp == nullptr)
     return fail(W4_ERR_NULL, "x, qw, scales and zp must not be NULL");
@@ -270,7 +279,7 @@ static w4_status matmul_one(const w4_desc& d, void* ws, size_t wsb, w4_path path
   const DeviceInfo* di = nullptr;
   rc = current_device(&di);
   if (rc != W4_OK) return rc;
-  if (d.K == 0) return launch_zero_fill(d.y, d.ldy, d.M, d.N, st);
+  if (d.K == 0) return launch_zero_fill(d.y, d.ldy, d.M, d.N, st, &d);
   const char* why = "";
   const char* why_tc = "";
   const bool gemv_ok = gemv_eligible(d, &why);
@@ -287,6 +296,11 @@ static w4_status matmul_one(const w4_desc& d, void* ws, size_t wsb, w4_path path
       if (d.M > kTcMinM) return tc_ok ? launch_tc(&d, 1, st, *di) : launch_generic(d, st, *di);
       return gemv_ok ? launch_gemv(&d, 1, ws, wsb, st, *di) : launch_generic(d, st, *di);
   }
+}
+
+w4_status w4_matmul_desc(const w4_desc* d, void* workspace, size_t workspace_bytes, w4_path path, void* stream) {
+  if (d == nullptr) return fail(W4_ERR_NULL, "descriptor is NULL");
+  return matmul_one(*d, workspace, workspace_bytes, path, static_cast<cudaStream_t>(stream));
 }
 
 w4_status w4_matmul_path(const float* x, int64_t ldx, const uint8_t* qw, const float* scales, const uint8_t* zp,
@@ -353,7 +367,7 @@ w4_status w4_matmul_grouped(const w4_desc* descs, int32_t count, void* workspace
     if (d.M == 0 || d.N == 0) continue;
     const char* why = "";
     if (d.K == 0) {
-      rc = launch_zero_fill(d.y, d.ldy, d.M, d.N, st);
+      rc = launch_zero_fill(d.y, d.ldy, d.M, d.N, st, &d);
     } else if (d.M > kTcMinM) {
       if (!tc_eligible(d, &why)) {
         rc = launch_generic(d, st, *di);

@@ -195,4 +195,39 @@ __device__ __forceinline__ float inv_slot_scale(int slot) {
   return slot == 0 ? 1.0f : (slot == 1 ? 0.0625f : (slot == 2 ? 0.00390625f : 0.000244140625f));
 }
 
+// ---------------------------------------------------------------- fused epilogue
+
+// y = act(v + bias[n]) + residual[m * ldr + n] (the MatMul + Add that the
+// export's gemm_to_matmul step leaves behind each GPT-2 weight, with the
+// activation or residual add that follows it in the model). Zero pointers /
+// W4_ACT_NONE switch the parts off. GELU forms as in include/w4.h; tanhf and
+// erff are CUDA's single-precision functions.
+struct Epi {
+  const float* bias;
+  const float* res;
+  int64_t ldr;
+  int32_t act;
+  int32_t pad;
+};
+
+__device__ __forceinline__ float gelu_tanh_f(float v) {
+  const float c0 = 0.7978845608028654f;  // sqrt(2 / pi)
+  const float c1 = 0.044715f;
+  return 0.5f * v * (1.f + tanhf(c0 * (v + c1 * v * v * v)));
+}
+
+__device__ __forceinline__ float gelu_erf_f(float v) { return 0.5f * v * (1.f + erff(v * 0.7071067811865476f)); }
+
+__device__ __forceinline__ bool epi_active(const Epi& e) {
+  return e.bias != nullptr || e.res != nullptr || e.act != W4_ACT_NONE;
+}
+
+__device__ __forceinline__ float epi_apply(float v, const Epi& e, int64_t m, int64_t n) {
+  if (e.bias != nullptr) v += e.bias[n];
+  if (e.act == W4_ACT_GELU_TANH) v = gelu_tanh_f(v);
+  else if (e.act == W4_ACT_GELU_ERF) v = gelu_erf_f(v);
+  if (e.res != nullptr) v += e.res[m * e.ldr + n];
+  return v;
+}
+
 }  // namespace w4dev

@@ -93,6 +93,7 @@ struct MatScalars {
   int32_t nnar;    // narrow tiles after them (the last may be partial)
   int32_t nmc;     // groups of MT rows
   int32_t pad;
+  Epi epi;         // fused epilogue of the final store
 };
 static_assert(sizeof(MatScalars) % 8 == 0, "copied as 8-byte words");
 constexpr int MS_WORDS = sizeof(MatScalars) / 8;
@@ -143,6 +144,7 @@ struct Cfg {
   static constexpr int BAR_OFF = SCAL_OFF + W4_GROUP_MAX * static_cast<int>(sizeof(MatScalars));
   static constexpr int NBARS = 2 * NSTAGES + 4;  // full, empty, red_full[2], red_empty[2]
   static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 64;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
 };
 
 // Flat unit f -> (matrix, tile, group of rows, unit within the tile).
@@ -582,12 +584,21 @@ __device__ __forceinline__ void finish_segment(const float* red, const SegInfo& 
           for (int i = 0; i < PER; ++i) v[i] += t[i];
         }
       }
-      float* yrow = m.y + static_cast<int64_t>(s.mc * MT + mm) * m.ldy + s.col0;
+      const int64_t row = static_cast<int64_t>(s.mc * MT + mm);
+      float* yrow = m.y + row * m.ldy + s.col0;
       const int ncol = min(s.wt, m.N - s.col0);
+      if (epi_active(m.epi)) {
 #pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        const int c = tid + i * NT;
-        if (c < ncol) yrow[c] = v[i];
+        for (int i = 0; i < PER; ++i) {
+          const int c = tid + i * NT;
+          if (c < ncol) yrow[c] = epi_apply(v[i], m.epi, row, s.col0 + c);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int c = tid + i * NT;
+          if (c < ncol) yrow[c] = v[i];
+        }
       }
     }
   }
@@ -1097,6 +1108,7 @@ w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cud
     m.y = s.y;
     m.ldx = s.ldx;
     m.ldy = s.ldy;
+    m.epi = Epi{s.bias, s.residual, s.ldr, s.act, 0};
     m.M = static_cast<int32_t>(s.M);
     m.K = static_cast<int32_t>(s.K);
     m.N = static_cast<int32_t>(s.N);

@@ -24,7 +24,7 @@ __global__ void __launch_bounds__(128) w4_generic_kernel(const float* __restrict
                                                          const uint8_t* __restrict__ qw,
                                                          const float* __restrict__ scales,
                                                          const uint8_t* __restrict__ zp, float* __restrict__ y,
-                                                         int64_t ldy, int64_t M, int64_t K, int64_t N) {
+                                                         int64_t ldy, int64_t M, int64_t K, int64_t N, Epi epi) {
   const int64_t pcol = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // column pair
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * GEN_MT;
   const int64_t half = N / 2;
@@ -75,16 +75,17 @@ __global__ void __launch_bounds__(128) w4_generic_kernel(const float* __restrict
 #pragma unroll
   for (int m = 0; m < GEN_MT; ++m) {
     if (m < mrows) {
-      y[(m0 + m) * ldy + 2 * pcol] = tot0[m];
-      y[(m0 + m) * ldy + 2 * pcol + 1] = tot1[m];
+      y[(m0 + m) * ldy + 2 * pcol] = epi_apply(tot0[m], epi, m0 + m, 2 * pcol);
+      y[(m0 + m) * ldy + 2 * pcol + 1] = epi_apply(tot1[m], epi, m0 + m, 2 * pcol + 1);
     }
   }
 }
 
-__global__ void zero_fill_kernel(float* y, int64_t ldy, int64_t M, int64_t N) {
+// y = 0 (K = 0), through the epilogue when one is given.
+__global__ void zero_fill_kernel(float* y, int64_t ldy, int64_t M, int64_t N, Epi epi) {
   const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t m = blockIdx.y;
-  if (n < N && m < M) y[m * ldy + n] = 0.f;
+  if (n < N && m < M) y[m * ldy + n] = epi_apply(0.f, epi, m, n);
 }
 
 // One thread per (token column, group of 8 rows of h).
@@ -148,15 +149,18 @@ w4_status launch_generic(const w4_desc& d, cudaStream_t st, const DeviceInfo&) {
   const int64_t half = d.N / 2;
   const dim3 grid(static_cast<unsigned>((half + 127) / 128), static_cast<unsigned>((d.M + GEN_MT - 1) / GEN_MT));
   if (grid.y > 65535) return fail(W4_ERR_SHAPE, "M too large for the generic kernel");
-  w4_generic_kernel<<<grid, 128, 0, st>>>(d.x, d.ldx, d.qw, d.scales, d.zp, d.y, d.ldy, d.M, d.K, d.N);
+  w4_generic_kernel<<<grid, 128, 0, st>>>(d.x, d.ldx, d.qw, d.scales, d.zp, d.y, d.ldy, d.M, d.K, d.N,
+                                          Epi{d.bias, d.residual, d.ldr, d.act, 0});
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? W4_OK : cuda_fail(e, "launch w4_generic");
 }
 
-w4_status launch_zero_fill(float* y, int64_t ldy, int64_t M, int64_t N, cudaStream_t st) {
+w4_status launch_zero_fill(float* y, int64_t ldy, int64_t M, int64_t N, cudaStream_t st, const w4_desc* epi_of) {
   if (M > 65535) return fail(W4_ERR_SHAPE, "M too large for the zero fill");
   const dim3 grid(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(M));
-  zero_fill_kernel<<<grid, 256, 0, st>>>(y, ldy, M, N);
+  const Epi epi = epi_of == nullptr ? Epi{nullptr, nullptr, 0, W4_ACT_NONE, 0}
+                                    : Epi{epi_of->bias, epi_of->residual, epi_of->ldr, epi_of->act, 0};
+  zero_fill_kernel<<<grid, 256, 0, st>>>(y, ldy, M, N, epi);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? W4_OK : cuda_fail(e, "launch zero_fill");
 }

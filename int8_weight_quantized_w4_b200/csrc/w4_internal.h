@@ -49,7 +49,9 @@ w4_status launch_generic(const w4_desc& d, cudaStream_t st, const DeviceInfo& di
 constexpr int64_t kTcMinM = 16;
 bool tc_eligible(const w4_desc& d, const char** why);
 w4_status launch_tc(const w4_desc* d, int count, cudaStream_t st, const DeviceInfo& di);
-w4_status launch_zero_fill(float* y, int64_t ldy, int64_t M, int64_t N, cudaStream_t st);
+// y = 0 for K = 0; with epi_of, through that descriptor's fused epilogue.
+w4_status launch_zero_fill(float* y, int64_t ldy, int64_t M, int64_t N, cudaStream_t st,
+                           const w4_desc* epi_of = nullptr);
 
 // ---- head kernels
 struct HeadArgs {

@@ -66,6 +66,7 @@ struct TcMat {
   int64_t ldx, ldy;
   int32_t M, K, N, nb;
   int32_t tiles_m, tile_off;  // tiles of this weight: tiles_m x ceil(N / BN), from tile_off on
+  Epi epi;                    // fused epilogue of the store
 };
 
 struct TcParams {
@@ -300,9 +301,15 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
       if (row < m.M) {
         float* yr = m.y + static_cast<int64_t>(row) * m.ldy + n0 + ch;
         const int ncol = m.N - n0;
+        if (epi_active(m.epi)) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (8 * i + ch < ncol) yr[8 * i] = __uint_as_float(v[i]);
+          for (int i = 0; i < 32; ++i)
+            if (8 * i + ch < ncol) yr[8 * i] = epi_apply(__uint_as_float(v[i]), m.epi, row, n0 + ch + 8 * i);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (8 * i + ch < ncol) yr[8 * i] = __uint_as_float(v[i]);
+        }
       }
     }
   }
@@ -349,6 +356,7 @@ w4_status launch_tc(const w4_desc* d, int count, cudaStream_t st, const DeviceIn
     m.y = s.y;
     m.ldx = s.ldx;
     m.ldy = s.ldy;
+    m.epi = Epi{s.bias, s.residual, s.ldr, s.act, 0};
     m.M = static_cast<int32_t>(s.M);
     m.K = static_cast<int32_t>(s.K);
     m.N = static_cast<int32_t>(s.N);

@@ -44,7 +44,7 @@ DENSE38_LAYER_SHAPES = (
     ("down", 8192, 3072),
 )
 
-_TAGS = {"w4": 1, "x": 2, "table": 3, "head_scales": 4, "h": 5, "misc": 6}
+_TAGS = {"w4": 1, "x": 2, "table": 3, "head_scales": 4, "h": 5, "misc": 6, "bias": 7}
 
 
 def generator(tag: str, *idx: int, seed: int = BASE_SEED) -> np.random.Generator:
@@ -71,6 +71,12 @@ def activations(M: int, K: int, *idx: int, seed: int = BASE_SEED, ld: int | None
     out = np.full((M, ld), np.nan, dtype=np.float32)
     out[:, :K] = x
     return out
+
+
+def bias(N: int, *idx: int, seed: int = BASE_SEED, std: float = 0.5) -> np.ndarray:
+    """fp32 N(0, std^2) vector [N] (a bias of the fused epilogue)."""
+    g = generator("bias", N, *idx, seed=seed)
+    return (std * g.standard_normal(size=N)).astype(np.float32)
 
 
 def i8_head(K: int, V: int, *idx: int, seed: int = BASE_SEED, ldt: int | None = None) -> dict:

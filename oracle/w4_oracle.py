@@ -30,12 +30,17 @@ Readings where the page is silent (each is listed in the design notes):
 * dequantisation is exact in (q - zp) and then one fp32 multiply rounded to
   nearest-even, which is what DequantizeLinear computes in fp32;
 * the head has no zero point (symmetric) and no bias.
+* the optional fused epilogue restores the Add that step 1 splits off, then
+  applies stock GPT-2's activation (the tanh form of GELU; the erf form is
+  offered too) or its residual add: out = act(y + bias) + residual.
 
 Accumulation is fp64. Every function also returns sum_k |x_k * w_kn| so that
 callers can apply the tolerance |y - y_ref| <= 1e-5 * sum|x*w| + 1e-6.
 """
 
 from __future__ import annotations
+
+import math
 
 import numpy as np
 
@@ -229,6 +234,52 @@ def last_position_rows(hidden, T: int, K: int) -> np.ndarray:
     """Rows T-1 of M sequences of hidden states [M, T, K] (last_token_logits)."""
     hs = np.asarray(hidden, dtype=np.float32).reshape(-1, T, K)
     return np.ascontiguousarray(hs[:, T - 1, :])
+
+
+# --------------------------------------------------------------------------
+# fused epilogue: the Add that gemm_to_matmul splits off, and what follows it
+# --------------------------------------------------------------------------
+# The page's step 1 turns every GPT-2 Conv1D into MatMul + Add (bias). The
+# model ("stock GPT-2 small") then applies GELU after the MLP's first weight
+# and adds the residual stream after the attention and MLP output weights.
+# Reading: GPT-2's activation is the tanh form of GELU ("gelu_new"); the erf
+# form (the exact GELU) is offered beside it. Order: act(y + bias) + residual.
+
+SQRT_2_OVER_PI = float(np.sqrt(2.0 / np.pi))
+GELU_TANH_CUBIC = 0.044715
+GELU_DERIV_MAX = 1.13  # max of d/dv GELU(v) over the reals (both forms): 1.1290 at v ~ 1.41
+
+
+def gelu_tanh(v) -> np.ndarray:
+    """0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), fp64."""
+    v = np.asarray(v, dtype=np.float64)
+    return 0.5 * v * (1.0 + np.tanh(SQRT_2_OVER_PI * (v + GELU_TANH_CUBIC * v ** 3)))
+
+
+def gelu_erf(v) -> np.ndarray:
+    """0.5 v (1 + erf(v / sqrt 2)) = v * Phi(v), fp64 (math.erf per element)."""
+    v = np.asarray(v, dtype=np.float64)
+    erf = np.vectorize(math.erf, otypes=[np.float64])
+    return 0.5 * v * (1.0 + erf(v / math.sqrt(2.0)))
+
+
+ACTIVATIONS = {"none": lambda v: np.asarray(v, dtype=np.float64), "gelu_tanh": gelu_tanh, "gelu_erf": gelu_erf}
+
+
+def epilogue_ref(y, a, bias=None, residual=None, act: str = "none"):
+    """out = act(y + bias) + residual in fp64 for y = x.W (fp64 [M, N]) with
+    its sum|x*w| a; returns (out, tol), tol the per-output allowance for an
+    fp32 kernel: the body's allowance carried through the activation's slope
+    (at most GELU_DERIV_MAX), plus a few fp32 roundings of the bias add, the
+    activation and the residual add (1e-6 relative to |pre| and |out|)."""
+    y = np.asarray(y, dtype=np.float64)
+    pre = y + (0.0 if bias is None else np.asarray(bias, dtype=np.float32).astype(np.float64)[None, :])
+    out = ACTIVATIONS[act](pre)
+    if residual is not None:
+        out = out + np.asarray(residual, dtype=np.float32).astype(np.float64)
+    slope = 1.0 if act == "none" else GELU_DERIV_MAX
+    tol = slope * tolerance(a) + 1e-6 * (np.abs(pre) + np.abs(out))
+    return out, tol
 
 
 # --------------------------------------------------------------------------

@@ -48,7 +48,8 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = _lib()
-    assert lib.w4_abi_version() == 1
+    from int8_weight_quantized_w4_b200 import _lib as L
+    assert lib.w4_abi_version() == L.ABI_VERSION == 2
     assert lib.w4_status_string(0) == b"W4_OK"
     assert lib.w4_status_string(6) == b"W4_ERR_TIMEOUT"
     assert lib.w4_status_string(99) == b"W4_ERR_UNKNOWN"
@@ -120,6 +121,51 @@ def test_grouped_argument_errors():
     assert b"descriptor 1" in lib.w4_last_error()
     assert lib.w4_matmul_grouped(d, 0, None, 0, None) == 0
     assert lib.w4_matmul_grouped(None, 3, None, 0, None) == 1
+
+
+def test_desc_layout_matches_the_c_struct(tmp_path):
+    """The ctypes descriptor has the C struct's size and field offsets."""
+    from int8_weight_quantized_w4_b200._lib import W4Desc
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "w4.h"\n'
+                   'int main(void) { printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(w4_desc), offsetof(w4_desc, N), '
+                   'offsetof(w4_desc, bias), offsetof(w4_desc, residual), offsetof(w4_desc, ldr), '
+                   'offsetof(w4_desc, act)); return 0; }\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    want = [C.sizeof(W4Desc), W4Desc.N.offset, W4Desc.bias.offset, W4Desc.residual.offset, W4Desc.ldr.offset,
+            W4Desc.act.offset]
+    assert got == want
+
+
+def _desc(**kw):
+    from int8_weight_quantized_w4_b200._lib import W4Desc
+    a = dict(x=0x1000, ldx=64, qw=0x2000, scales=0x3000, zp=0x4000, y=0x5000, ldy=64, M=1, K=64, N=64, bias=0,
+             residual=0, ldr=0, act=0, reserved=0)
+    a.update(kw)
+    return W4Desc(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(act=3), 8), (dict(act=-1), 8), (dict(reserved=1), 8),
+    (dict(bias=0x6002), 3), (dict(residual=0x7002, ldr=64), 3),
+    (dict(residual=0x7000, ldr=32), 2), (dict(residual=0x5000, ldr=128), 2),
+    (dict(K=40), 2), (dict(y=0), 1),
+])
+def test_epilogue_argument_errors_before_any_launch(kw, status):
+    lib = _lib()
+    d = _desc(**kw)
+    assert lib.w4_matmul_desc(C.byref(d), None, 0, 0, None) == status
+    assert lib.w4_last_error()
+    g = (type(d) * 1)(d)
+    assert lib.w4_matmul_grouped(g, 1, None, 0, None) == status
+
+
+def test_epilogue_noops_need_no_device():
+    lib = _lib()
+    assert lib.w4_matmul_desc(C.byref(_desc(M=0, act=1, bias=0x6000)), None, 0, 0, None) == 0
+    assert lib.w4_matmul_desc(None, None, 0, 0, None) == 1
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
