@@ -251,6 +251,39 @@ W4_API w4_status i8_head_argmax(const float* h, int64_t ldh, const int8_t* table
 W4_API w4_status i8_embed_lookup(const int8_t* table, int64_t ldt, const float* scales, const int32_t* tokens,
                                  int64_t ntok, float* out, int64_t ldo, int64_t K, int64_t V, void* stream);
 
+/* ------------------------------------------------------------------ quantisers */
+
+/* Scale storage of w4_quantize: fp32 (the shipped format, the one every
+ * matmul here reads) or fp16 (the "fp16 scales" variant the page measures;
+ * widen it to fp32, exactly, before a matmul). */
+typedef enum w4_scale_type { W4_SCALE_F32 = 0, W4_SCALE_F16 = 1 } w4_scale_type;
+
+/* The export's dq4 step ("ONNX export, quantization and the browser
+ * runtime", section "Quantization (train/quantize.py)", step 2) on the GPU:
+ * w [K, N] fp32 (row stride ldw >= N, 4-byte aligned, finite values) ->
+ *   qw [K*N/2] packed nibbles (flat [K, N] order, low nibble first),
+ *   scales [K/block, N] (fp32, or fp16 with W4_SCALE_F16; aligned to the
+ *   element size), zp [(K/block)*N/2] packed nibbles.
+ * block is 32 (the shipped format) or 64 (the group size of the page's MLX
+ * comparison); K % block == 0 and N even (else W4_ERR_SHAPE / W4_ERR_VALUE).
+ * The page gives no formula; this is the min/max reading, in fp64 with one
+ * rounding per division: lo = min(min w, 0) and hi = max(max w, 0) over the
+ * block of one column; s = (hi - lo) / 15 rounded once to the stored type;
+ * a stored s of 0 becomes s = 1, zp = 0; zp = rint(-lo / s) and
+ * q = rint(w / s) + zp, clamped to 0..15, rint rounding half to even.
+ * Buffers are the caller's device memory; the call is asynchronous and
+ * stream-ordered. */
+W4_API w4_status w4_quantize(const float* w, int64_t ldw, int64_t K, int64_t N, int32_t block, int32_t scale_type,
+                             uint8_t* qw, void* scales, uint8_t* zp, void* stream);
+
+/* The export's embedding_int8 step (same section, step 3) on the GPU:
+ * w [K, V] fp32 (row stride ldw >= V) -> table [K, V] int8 (row stride
+ * ldt >= V) and scales [V] fp32, one per token (column): in fp64,
+ * s = max|w| / 127 rounded once to fp32 (an all-zero column takes s = 1),
+ * q = rint(w / s) clamped to -127..127. */
+W4_API w4_status i8_quantize_head(const float* w, int64_t ldw, int64_t K, int64_t V, int8_t* table, int64_t ldt,
+                                  float* scales, void* stream);
+
 /* ------------------------------------------------------------------ host packing */
 
 /* Pack n uint4 values (each 0..15) into (n + 1) / 2 bytes, low nibble first;

@@ -10,6 +10,8 @@ Operations (see include/w4.h for layouts and error behaviour):
       (..., bias=, residual=, act=)         y = act(x . W + bias) + residual, fused
   w4_matmul_grouped([...])                  many independent ones, one launch
   i8_head_logits(h, table, scales, K, V)    last-position logits, int8 head
+  w4_quantize(w, block, scale_type)         the dq4 quantiser (GPU)
+  i8_quantize_head(w)                       the embedding_int8 quantiser (GPU)
   pack_nibbles / unpack_nibbles             host-side UINT4 packing
 """
 
@@ -224,6 +226,44 @@ def i8_embed_lookup(table, scales, tokens, K: int, V: int, ldt: int | None = Non
                                _stream_handle(stream))
     _check(st, "i8_embed_lookup")
     return out
+
+
+# ---------------------------------------------------------------- quantisers
+
+SCALE_TYPES = {"fp32": 0, "fp16": 1}
+
+
+def w4_quantize(w, block: int = 32, scale_type: str = "fp32", stream=None):
+    """The export's dq4 step on the GPU: fp32 w [K, N] -> (qw [K*N/2] uint8,
+    scales [K/block, N] fp32 or fp16, zp [(K/block)*N/2] uint8)."""
+    torch = _torch()
+    if w.dim() != 2 or w.dtype != torch.float32:
+        raise ValueError("w must be a 2-D fp32 tensor")
+    if scale_type not in SCALE_TYPES:
+        raise ValueError(f"scale_type must be one of {sorted(SCALE_TYPES)}")
+    K, N = w.shape
+    nb = K // block if block > 0 else 0
+    qw = torch.empty(K * N // 2, dtype=torch.uint8, device=w.device)
+    sc = torch.empty((nb, N), dtype=torch.float32 if scale_type == "fp32" else torch.float16, device=w.device)
+    zp = torch.empty(nb * N // 2, dtype=torch.uint8, device=w.device)
+    st = lib().w4_quantize(_ptr(w), _ld(w, N), K, N, block, SCALE_TYPES[scale_type], _ptr(qw), _ptr(sc), _ptr(zp),
+                           _stream_handle(stream))
+    _check(st, "w4_quantize")
+    return qw, sc, zp
+
+
+def i8_quantize_head(w, stream=None):
+    """The export's embedding_int8 step on the GPU: fp32 w [K, V] ->
+    (table [K, V] int8, scales [V] fp32)."""
+    torch = _torch()
+    if w.dim() != 2 or w.dtype != torch.float32:
+        raise ValueError("w must be a 2-D fp32 tensor")
+    K, V = w.shape
+    table = torch.empty((K, V), dtype=torch.int8, device=w.device)
+    sc = torch.empty(V, dtype=torch.float32, device=w.device)
+    st = lib().i8_quantize_head(_ptr(w), _ld(w, V), K, V, _ptr(table), V, _ptr(sc), _stream_handle(stream))
+    _check(st, "i8_quantize_head")
+    return table, sc
 
 
 # ---------------------------------------------------------------- host packing

@@ -74,6 +74,10 @@ SIGNATURES = {
     "i8_head_logits_path": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
                                       C.c_int64, C.c_int64, C.c_int64, C.c_int64, C.c_void_p, C.c_size_t, C.c_int,
                                       C.c_void_p]),
+    "w4_quantize": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.c_int32, C.c_int32, C.c_void_p,
+                              C.c_void_p, C.c_void_p, C.c_void_p]),
+    "i8_quantize_head": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p,
+                                   C.c_void_p]),
     "w4_pack_nibbles": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p]),
     "w4_unpack_nibbles": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p]),
     "w4_status_string": (C.c_char_p, [C.c_int]),

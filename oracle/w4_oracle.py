@@ -45,6 +45,7 @@ import math
 import numpy as np
 
 BLOCK = 32  # K-block length of the 4-bit format (dq4: "blocks of 32 along K")
+QUANT_BLOCKS = (32, 64)  # the shipped block, and the group of 64 the page's MLX comparison uses
 ABS_TOL = 1e-6
 REL_TOL = 1e-5
 
@@ -96,28 +97,31 @@ def _rows(x, K: int) -> np.ndarray:
     return a.astype(np.float64)
 
 
-def check_w4_shape(K: int, N: int) -> None:
+def check_w4_shape(K: int, N: int, block: int = BLOCK) -> None:
     if K < 0 or N < 0:
         raise ValueError("negative shape")
-    if K % BLOCK:
-        raise ValueError(f"K={K} is not a multiple of {BLOCK}")
+    if block not in QUANT_BLOCKS:
+        raise ValueError(f"block {block} is not one of {QUANT_BLOCKS}")
+    if K % block:
+        raise ValueError(f"K={K} is not a multiple of {block}")
     if N % 2:
         raise ValueError(f"N={N} is odd")
 
 
-def dequantize_w4(qw, scales, zp, K: int, N: int) -> np.ndarray:
+def dequantize_w4(qw, scales, zp, K: int, N: int, block: int = BLOCK) -> np.ndarray:
     """Blocked DequantizeLinear of one [K, N] weight: fp32 w = (q - zp) * s.
 
     ``qw`` holds K*N packed nibbles (flat [K, N] order), ``zp`` holds
-    (K/32)*N packed nibbles (flat [K/32, N] order) and ``scales`` is fp32
-    [K/32, N]. Row k uses block b = k // 32.
+    (K/block)*N packed nibbles (flat [K/block, N] order) and ``scales`` is
+    [K/block, N], fp32 (or fp16, widened exactly). Row k uses block
+    b = k // block; the shipped format has block = 32.
     """
-    check_w4_shape(K, N)
-    nb = K // BLOCK
+    check_w4_shape(K, N, block)
+    nb = K // block
     q = unpack_nibbles(qw, K * N).reshape(K, N).astype(np.int32)
     z = unpack_nibbles(zp, nb * N).reshape(nb, N).astype(np.int32)
-    s = np.ascontiguousarray(scales, dtype=np.float32).reshape(nb, N)
-    blk = np.arange(K) // BLOCK
+    s = np.ascontiguousarray(scales).astype(np.float32).reshape(nb, N)
+    blk = np.arange(K) // block
     diff = (q - z[blk, :]).astype(np.float32)  # small integers: exact in fp32
     return diff * s[blk, :]  # one fp32 multiply, round to nearest even
 
@@ -303,28 +307,41 @@ def max_violation(y, y_ref, a) -> float:
 
 
 # --------------------------------------------------------------------------
-# quantisers (self-checks of the oracle only; not on the product path)
+# quantisers: the export's dq4 (step 2) and embedding_int8 (step 3), the
+# reference of the GPU quantisers and of the oracle's own self-checks
 # --------------------------------------------------------------------------
 
-def quantize_w4(w) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
-    """Asymmetric min/max 4-bit quantiser, per (32-row block, column).
+def stored_scale(s64, scale_type: str):
+    """The stored form of a scale computed in fp64: fp32 (the shipped format)
+    or fp16 (the page's "fp16 scales" variant), one round-to-nearest-even."""
+    return np.asarray(s64, dtype=np.float64).astype(np.float16 if scale_type == "fp16" else np.float32)
+
+
+def quantize_w4(w, block: int = BLOCK, scale_type: str = "fp32") -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Asymmetric min/max 4-bit quantiser, per (block of rows, column).
 
     The page says "asymmetric, blocks of 32 along K" and gives no formula; this
-    is the plainest min/max reading: the range [lo, hi] always contains 0,
-    s = (hi - lo) / 15 stored as fp32, zp = rint(-lo / s) clamped to 0..15,
-    q = rint(w / s) + zp clamped to 0..15 (rint rounds half to even). A block
-    with hi == lo (all zeros) takes s = 1, zp = 0.
-    Returns packed qw, fp32 scales [K/32, N], packed zp.
+    is the plainest min/max reading, every step in fp64 (the differences of
+    fp32 values are exact there, and each division rounds once):
+      lo = min(min w, 0), hi = max(max w, 0) over the block (and column);
+      s = (hi - lo) / 15, rounded once to the stored type (fp32 or fp16);
+      a block whose stored s is 0 (all zeros, or a range below the type's
+      smallest value) takes s = 1, zp = 0;
+      zp = rint(-lo / s), q = rint(w / s) + zp, both clamped to 0..15, with
+      s the stored value and rint rounding half to even.
+    Returns packed qw, scales [K/block, N] of the stored type, packed zp.
     """
+    if scale_type not in ("fp32", "fp16"):
+        raise ValueError(f"scale_type {scale_type!r}")
     w = np.asarray(w, dtype=np.float32)
     K, N = w.shape
-    check_w4_shape(K, N)
-    nb = K // BLOCK
-    wb = w.astype(np.float64).reshape(nb, BLOCK, N)
+    check_w4_shape(K, N, block)
+    nb = K // block
+    wb = w.astype(np.float64).reshape(nb, block, N)
     lo = np.minimum(wb.min(axis=1), 0.0)
     hi = np.maximum(wb.max(axis=1), 0.0)
-    s = ((hi - lo) / 15.0).astype(np.float32)
-    flat = hi == lo
+    s = stored_scale((hi - lo) / 15.0, scale_type)
+    flat = s == 0
     s[flat] = 1.0
     s64 = s.astype(np.float64)
     zp = np.clip(np.rint(-lo / s64), 0, 15)
@@ -335,12 +352,13 @@ def quantize_w4(w) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
 
 
 def quantize_i8_head(w) -> tuple[np.ndarray, np.ndarray]:
-    """Symmetric int8 quantiser, one scale per column (token) of [K, V]:
-    s = max|w| / 127, q = rint(w / s) clamped to -127..127; an all-zero
-    column takes s = 1."""
+    """Symmetric int8 quantiser, one scale per column (token) of [K, V]
+    (the page's embedding_int8: "int8 with one scale per token"), in fp64:
+    s = max|w| / 127 rounded once to fp32, q = rint(w / s) clamped to
+    -127..127; a column whose s is 0 (all zeros) takes s = 1."""
     w = np.asarray(w, dtype=np.float32)
     amax = np.abs(w.astype(np.float64)).max(axis=0)
     s = (amax / 127.0).astype(np.float32)
-    s[amax == 0] = 1.0
+    s[s == 0] = 1.0
     q = np.clip(np.rint(w.astype(np.float64) / s.astype(np.float64)[None, :]), -127, 127)
     return q.astype(np.int8), s

@@ -168,6 +168,29 @@ def test_epilogue_noops_need_no_device():
     assert lib.w4_matmul_desc(None, None, 0, 0, None) == 1
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(block=48), 8), (dict(block=0), 8), (dict(st=2), 8), (dict(K=96, block=64), 2), (dict(N=63), 2),
+    (dict(ldw=32), 2), (dict(w=0), 1), (dict(qw=0), 1), (dict(w=0x1002), 3), (dict(sc=0x3002), 3),
+    (dict(sc=0x3001, st=1), 3), (dict(K=-64), 2),
+])
+def test_quantize_argument_errors_before_any_launch(kw, status):
+    lib = _lib()
+    a = dict(w=0x1000, ldw=64, K=128, N=64, block=32, st=0, qw=0x2000, sc=0x3000, zp=0x4000)
+    a.update(kw)
+    assert lib.w4_quantize(a["w"], a["ldw"], a["K"], a["N"], a["block"], a["st"], a["qw"], a["sc"], a["zp"],
+                           None) == status
+    assert lib.w4_last_error()
+
+
+def test_quantize_head_argument_errors_before_any_launch():
+    lib = _lib()
+    assert lib.i8_quantize_head(0x1000, 10, 8, 20, 0x2000, 20, 0x3000, None) == 2   # ldw < V
+    assert lib.i8_quantize_head(0x1000, 20, 8, 20, 0x2000, 10, 0x3000, None) == 2   # ldt < V
+    assert lib.i8_quantize_head(0x1002, 20, 8, 20, 0x2000, 20, 0x3000, None) == 3
+    assert lib.i8_quantize_head(0x1000, 20, 8, 20, 0x2000, 20, 0, None) == 1
+    assert lib.i8_quantize_head(0x1000, 20, 8, 0, 0x2000, 20, 0x3000, None) == 0    # V = 0: nothing to do
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     from int8_weight_quantized_w4_b200 import _lib as L
     monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "nope.so"))
