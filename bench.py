@@ -200,10 +200,24 @@ class Workload:
         H = synth.i8_head(HEAD_K, HEAD_V, seed=seed)
         self.x_host = [synth.activations(1, K, i, seed=seed) for i, (_, K, _) in enumerate(self.shapes)]
         self.h_host = synth.activations(1, HEAD_K, 999, seed=seed)
-        self.xs = [torch.from_numpy(x).to(dev) for x in self.x_host]
-        self.h = torch.from_numpy(self.h_host).to(dev)
-        self.ys = [torch.empty((1, N), dtype=torch.float32, device=dev) for _, _, N in self.shapes]
-        self.logits = torch.empty((1, HEAD_V), dtype=torch.float32, device=dev)
+        # every input row (the 48 x and the head's h) in one device buffer, every
+        # output (the 48 y and the logits) in another, so that a step's inputs
+        # and outputs each cross PCIe in one copy; every row starts 16-byte aligned
+        self.in_host = np.concatenate([x.reshape(-1) for x in self.x_host] + [self.h_host.reshape(-1)])
+        self.in_dev = torch.from_numpy(self.in_host).to(dev)
+        self.xs, off = [], 0
+        for _, K, _ in self.shapes:
+            self.xs.append(self.in_dev[off:off + K].view(1, K))
+            off += K
+        self.h = self.in_dev[off:off + HEAD_K].view(1, HEAD_K)
+        n_out = sum(N for _, _, N in self.shapes) + HEAD_V
+        self.out_dev = torch.empty(n_out, dtype=torch.float32, device=dev)
+        self.ys, off = [], 0
+        for _, _, N in self.shapes:
+            self.ys.append(self.out_dev[off:off + N].view(1, N))
+            off += N
+        self.logits = self.out_dev[off:off + HEAD_V].view(1, HEAD_V)
+        assert all(t.data_ptr() % 16 == 0 for t in self.xs + self.ys + [self.h, self.logits])
         base = [{k: torch.from_numpy(W[k]).to(dev) for k in ("qw", "scales", "zp")} for W in host_w]
         table = torch.from_numpy(H["table"]).to(dev)
         hsc = torch.from_numpy(H["scales"]).to(dev)
@@ -375,22 +389,16 @@ def run_e2e(wl, args, world, R):
     import torch
     stream = torch.cuda.current_stream()
     sh = int(stream.cuda_stream)
-    xh = [torch.from_numpy(x).pin_memory() for x in wl.x_host]
-    hh = torch.from_numpy(wl.h_host).pin_memory()
-    yh = [torch.empty(y.shape, dtype=torch.float32).pin_memory() for y in wl.ys]
-    lh = torch.empty(wl.logits.shape, dtype=torch.float32).pin_memory()
-    h2d = sum(x.numel() * 4 for x in xh) + hh.numel() * 4
-    d2h = sum(y.numel() * 4 for y in yh) + lh.numel() * 4
+    inh = torch.from_numpy(wl.in_host).pin_memory()  # the 48 x and h, contiguous
+    outh = torch.empty(wl.out_dev.shape, dtype=torch.float32).pin_memory()  # the 48 y and the logits
+    h2d = inh.numel() * 4
+    d2h = outh.numel() * 4
 
     def step(r):
-        for d, s in zip(wl.xs, xh):
-            d.copy_(s, non_blocking=True)
-        wl.h.copy_(hh, non_blocking=True)
+        wl.in_dev.copy_(inh, non_blocking=True)
         wl.body(r, sh)
         wl.head(r, sh)
-        for d, s in zip(yh, wl.ys):
-            d.copy_(s, non_blocking=True)
-        lh.copy_(wl.logits, non_blocking=True)
+        outh.copy_(wl.out_dev, non_blocking=True)
 
     for i in range(3):
         step(i % R)

@@ -51,6 +51,10 @@
 //    the scale is applied once per slice (s * sum x (q - zp)).
 //    MT >= 2: the weight is dequantised to fp32 exactly as the oracle does
 //    ((q - zp) * s, one rounding) and reused for the MT rows of x.
+//  * The walk over segments (locate, seg_init, seg_next, seg_info) is inlined
+//    into each warp role: at kernel start a call into not-yet-fetched code
+//    costs about a microsecond of instruction fetch, and these calls sit on
+//    the producer's path to its first copy.
 //  * Accumulation is per 16-row slice, then across stages, then across
 //    warps, then across CTAs: all fp32, all in a fixed order.
 #include <cuda_runtime.h>
@@ -158,7 +162,7 @@ struct Pos {
 };
 
 // g is a matrix at or before the one holding f; g_hi the last this CTA touches.
-__device__ __noinline__ Pos locate(const MatScalars* ms, int g_hi, int64_t f, int g) {
+__device__ __forceinline__ Pos locate(const MatScalars* ms, int g_hi, int64_t f, int g) {
 #pragma unroll 1
   while (g < g_hi && ms[g + 1].u_off <= f) ++g;
   const MatScalars& m = ms[g];
@@ -214,7 +218,7 @@ struct SegIter {
   int g1, gm;        // last matrix of the range; cursor hint
 };
 
-__device__ __noinline__ void seg_init(SegIter& it, const MatScalars* ms, int g0, int g1, int64_t lo, int64_t hi,
+__device__ __forceinline__ void seg_init(SegIter& it, const MatScalars* ms, int g0, int g1, int64_t lo, int64_t hi,
                                       int fin) {
   it.lo = lo;
   it.hi = hi;
@@ -237,7 +241,7 @@ __device__ __noinline__ void seg_init(SegIter& it, const MatScalars* ms, int g0,
   it.f = it.hd_end;
 }
 
-__device__ __noinline__ bool seg_next(SegIter& it, const MatScalars* ms, int64_t& a, int64_t& b) {
+__device__ __forceinline__ bool seg_next(SegIter& it, const MatScalars* ms, int64_t& a, int64_t& b) {
   if (it.hd_end == it.hi) {  // a single segment
     if (it.k++ > 0) return false;
     a = it.lo;
@@ -363,7 +367,7 @@ __device__ __forceinline__ void stage_items(const uint8_t* st, int u, int n, int
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           wl[t] = item.q32[(r + t) * QS];
-          wh[t] = wl[t] >> 16;
+          wh[t] = __umulhi(wl[t], 65536u);  // = wl >> 16, issued on the FMA pipe, not the integer ALU
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -445,7 +449,7 @@ struct SegInfo {
 };
 
 // a: first unit of the segment; lo: first unit of this CTA's range; fin: its role bits.
-__device__ __noinline__ SegInfo seg_info(const MatScalars* ms, const Pos& ps, int64_t a, int64_t lo, int fin,
+__device__ __forceinline__ SegInfo seg_info(const MatScalars* ms, const Pos& ps, int64_t a, int64_t lo, int fin,
                                          int64_t W, int64_t G) {
   SegInfo s;
   s.m = &ms[ps.g];
