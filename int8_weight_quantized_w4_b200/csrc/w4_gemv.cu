@@ -61,6 +61,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <memory>
 #include <vector>
 
 #include "w4_device.cuh"
@@ -1080,8 +1081,49 @@ bool gemv_eligible(const w4_desc& d, const char** why) {
 
 size_t gemv_workspace_bytes(const w4_desc* d, int count, int sms) { return ws_bytes(make_plan(d, count, sms)); }
 
+// Launch parameters of recent calls, per host thread. A decode loop calls with
+// the same descriptors (weights, inputs and outputs at the same addresses)
+// every step; the parameters are a function of the descriptor bytes, the
+// workspace address and the device alone, so an exact match reuses them and
+// skips the tiling, the tensor-map lookups and the role assignment.
+struct PlanEntry {
+  int dev = -1;
+  int count = 0;
+  const void* ws = nullptr;
+  size_t need = 0;
+  int grid = 0;
+  int mt = 0;
+  uint64_t used = 0;
+  w4_desc descs[W4_GROUP_MAX];
+  GemvParams prm;
+};
+constexpr int kPlanEntries = 4;
+
+w4_status launch_planned(const PlanEntry& e, cudaStream_t st, const DeviceInfo& di) {
+  switch (e.mt) {
+    case 1: return launch_mt<1>(e.prm, e.grid, st, di);
+    case 2: return launch_mt<2>(e.prm, e.grid, st, di);
+    case 4: return launch_mt<4>(e.prm, e.grid, st, di);
+    default: return launch_mt<8>(e.prm, e.grid, st, di);
+  }
+}
+
 w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cudaStream_t st, const DeviceInfo& di) {
   if (count > W4_GROUP_MAX) return fail(W4_ERR_SHAPE, "at most %d matrices per GEMV launch", W4_GROUP_MAX);
+  static thread_local std::unique_ptr<PlanEntry[]> owned;  // kPlanEntries entries of ~37 KB, host memory
+  static thread_local uint64_t clock = 0;
+  if (!owned) owned.reset(new PlanEntry[kPlanEntries]);
+  PlanEntry* cache = owned.get();
+  ++clock;
+  for (int i = 0; i < kPlanEntries; ++i) {
+    PlanEntry& e = cache[i];
+    if (e.dev == di.dev && e.count == count && e.ws == ws && std::memcmp(e.descs, d, sizeof(w4_desc) * count) == 0) {
+      if (ws_size < e.need) return fail(W4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", e.need, ws_size);
+      e.used = clock;
+      e.prm.timeout_ns = wait_timeout_ns();
+      return launch_planned(e, st, di);
+    }
+  }
   const Plan pl = make_plan(d, count, di.sms);
   if (pl.W == 0) return W4_OK;
   // the kernel's flat-index arithmetic is 32-bit: W * grid must stay below 2^32
@@ -1094,7 +1136,12 @@ w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cud
   if ((reinterpret_cast<uintptr_t>(ws) & 15) != 0) return fail(W4_ERR_WORKSPACE, "workspace must be 16-byte aligned");
 
   static_assert(sizeof(GemvParams) <= 32000, "kernel parameters must fit the 32 KB limit");
-  static thread_local GemvParams prm;  // ~31 KB: kept off the host stack
+  int victim = 0;  // least recently used entry
+  for (int i = 1; i < kPlanEntries; ++i)
+    if (cache[i].used < cache[victim].used) victim = i;
+  PlanEntry& ent = cache[victim];
+  ent.dev = -1;  // invalid until the parameters are complete
+  GemvParams& prm = ent.prm;
   std::memset(&prm, 0, sizeof(prm));
   int g = 0;
   int64_t uoff = 0;
@@ -1162,12 +1209,15 @@ w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cud
   prm.ws_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + COUNTER_BYTES);
   prm.err = di.err;
   prm.timeout_ns = wait_timeout_ns();
-  switch (pl.mt) {
-    case 1: return launch_mt<1>(prm, pl.grid, st, di);
-    case 2: return launch_mt<2>(prm, pl.grid, st, di);
-    case 4: return launch_mt<4>(prm, pl.grid, st, di);
-    default: return launch_mt<8>(prm, pl.grid, st, di);
-  }
+  ent.count = count;
+  ent.ws = ws;
+  ent.need = need;
+  ent.grid = pl.grid;
+  ent.mt = pl.mt;
+  ent.used = clock;
+  std::memcpy(ent.descs, d, sizeof(w4_desc) * count);
+  ent.dev = di.dev;
+  return launch_planned(ent, st, di);
 }
 
 }  // namespace w4host
