@@ -474,6 +474,16 @@ def _oracle_step(ops, sel=None) -> int:
     return done
 
 
+def _cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(budget_s: float) -> dict:
     """The oracle, as it stands, on this host's cores: whole decode steps of
     the same workload (48 weights + head), repeated until ~budget_s (inputs
@@ -489,7 +499,8 @@ def cpu_baseline(budget_s: float) -> dict:
             break
     per_step = el / steps
     return {"value": round((body_bytes() + head_bytes()) / per_step / 1e9, 4), "unit": "GB/s",
-            "tokens_per_s": round(1 / per_step, 3), "cores": _blas_threads(), "kind": "oracle",
+            "tokens_per_s": round(1 / per_step, 3), "cores": _blas_threads(), "nproc": os.cpu_count(),
+            "cpu_model": _cpu_model(), "kind": "oracle",
             "sample": f"{steps} full decode steps (48 weights + head), {el:.1f} s; numpy unpack/dequantize "
                       f"single-threaded, fp64 matmul on BLAS threads"}
 
@@ -526,7 +537,8 @@ def run_reference(args, world, rank):
     sample = (f"{K} full decode steps (48 weights + head) on the host" if per_step == nops else
               f"{K} steps of {per_step} of the 49 ops each (48 weights + head, round-robin), "
               f"{done / 1e9:.2f} GB of weights in {el:.1f} s on the host")
-    cb = {"value": round(val, 4), "unit": "GB/s", "cores": _blas_threads(), "kind": "oracle", "sample": sample}
+    cb = {"value": round(val, 4), "unit": "GB/s", "cores": _blas_threads(), "nproc": os.cpu_count(),
+          "cpu_model": _cpu_model(), "kind": "oracle", "sample": sample}
     step_ms = (body_bytes() + head_bytes()) / (val * 1e9) * 1e3  # a whole step at the measured rate
     return {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": warm, "ms_per_step": round(step_ms, 3), "higher_is_better": True,
