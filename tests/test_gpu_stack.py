@@ -1,6 +1,7 @@
 """GPU parity of the decoder-stack workloads: the 48 GPT-2 weights in one
 grouped launch (decode M=1 and prefill M=58 followed by the head on the last
-row), and one layer of the 3.8B-dense stack at full size (sampled outputs)."""
+row), and one layer of the 3.8B-dense stack at full size (sampled outputs),
+as decode (M = 1, 8, 32) and as prefill (M = 2048)."""
 
 import numpy as np
 import pytest
@@ -101,7 +102,7 @@ def _sample_idx(g, M, N, K, n=4096):
     return rows, cols
 
 
-@pytest.mark.parametrize("M", [1, 8, 32])
+@pytest.mark.parametrize("M", [1, 8, 32, 2048])  # decode sizes, and the prefill size (tensor cores)
 def test_config4_dense38_one_layer_full_size_sampled(M):
     shapes = synth.dense38_stack_shapes()[:4]
     host, items = _stack(shapes, M, seed=31)
