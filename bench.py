@@ -227,10 +227,14 @@ class Workload:
             items = [{"x": self.xs[i], "y": self.ys[i], "K": K, "N": N, **ws[i]}
                      for i, (_, K, N) in enumerate(self.shapes)]
             descs = w4.make_descs(items)
+            # the same weights in the streaming layout (repacked once, at load)
+            wrs = [w4.w4_repack(d["qw"], d["scales"], d["zp"], K, N) for d, (_, K, N) in zip(ws, self.shapes)]
+            rdescs = w4.make_rdescs([{"x": self.xs[i], "y": self.ys[i], "K": K, "N": N, "wr": wrs[i]}
+                                     for i, (_, K, N) in enumerate(self.shapes)])
             t = table if r == 0 else table.clone()
             s = hsc if r == 0 else hsc.clone()
             # the descriptors hold raw pointers: keep every tensor they name alive
-            self.copies.append((descs, t, s, ws))
+            self.copies.append((descs, t, s, ws, rdescs, wrs))
         need = max(w4.w4_matmul_grouped_workspace_size(self.copies[0][0]),
                    w4.i8_head_workspace_size(1, HEAD_K, HEAD_V))
         self.ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
@@ -239,13 +243,21 @@ class Workload:
         torch.cuda.synchronize()
 
     def body(self, r: int, stream_handle: int):
+        """The 48 weights, repacked, in grouped decode launches (the product path)."""
+        rdescs = self.copies[r][4]
+        st = self.lib.w4r_matmul_grouped(rdescs, len(rdescs), stream_handle)
+        if st != 0:
+            raise RuntimeError(f"w4r_matmul_grouped failed: {st} {self.lib.w4_last_error()}")
+
+    def body_page_format(self, r: int, stream_handle: int):
+        """The same 48 weights in the page format through the split-K GEMV."""
         descs = self.copies[r][0]
         st = self.lib.w4_matmul_grouped(descs, len(descs), self.ws.data_ptr(), self.ws_bytes, stream_handle)
         if st != 0:
             raise RuntimeError(f"w4_matmul_grouped failed: {st} {self.lib.w4_last_error()}")
 
     def head(self, r: int, stream_handle: int):
-        _, t, s, _ = self.copies[r]
+        _, t, s = self.copies[r][:3]
         st = self.lib.i8_head_logits(self.h.data_ptr(), HEAD_K, t.data_ptr(), HEAD_V, s.data_ptr(),
                                      self.logits.data_ptr(), HEAD_V, 1, HEAD_K, HEAD_V, self.ws.data_ptr(),
                                      self.ws_bytes, stream_handle)
@@ -295,31 +307,46 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         return g
 
-    def timed(g):
+    def timed(g, reps=1):
+        """ms of `reps` back-to-back replays of g (K steps each)."""
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize()
         with torch.cuda.stream(side):
             t0.record(side)
-            g.replay()
+            for _ in range(reps):
+                g.replay()
             t1.record(side)
         torch.cuda.synchronize()
         barrier(world)
         return t0.elapsed_time(t1)
 
+    def reps_for(g, seconds):
+        """Replays of g that fill about `seconds` (from one untimed replay);
+        the same on every rank."""
+        one = max_over_ranks(timed(g), world)
+        return max(1, int(round(seconds * 1e3 / max(one, 1e-3))))
+
     g_step = capture([wl.body, wl.head])
     g_body = capture([wl.body])
     g_head = capture([wl.head])
+    g_page = capture([wl.body_page_format])
+    n_step = reps_for(g_step, args.seconds)
+    n_body = reps_for(g_body, args.seconds / 2)
+    n_head = reps_for(g_head, args.seconds / 2)
+    n_page = reps_for(g_page, args.seconds / 4)
     sampler = ClockSampler(gpu_id(local if world > 1 else 0))
     sampler.start()
     time.sleep(0.2)
-    total_ms = max_over_ranks(timed(g_step), world)
-    body_avg = timed(g_body) / K
-    head_avg = timed(g_head) / K
+    total_ms = max_over_ranks(timed(g_step, n_step), world)
+    body_avg = timed(g_body, n_body) / (K * n_body)
+    head_avg = timed(g_head, n_head) / (K * n_head)
+    page_avg = timed(g_page, n_page) / (K * n_page)
     clocks = sampler.stop()
-    ms_step = total_ms / K
-    del g_step, g_body, g_head
+    steps_timed = K * n_step
+    ms_step = total_ms / steps_timed
+    del g_step, g_body, g_head, g_page
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(wl, args, world, R)
@@ -333,7 +360,9 @@ def run_ours(args, world, rank, local):
         "value": round(value, 2),
         "unit": "GB/s",
         "n_gpus": n,
-        "steps": K,
+        "steps": steps_timed,
+        "steps_per_graph": K,
+        "graph_replays": n_step,
         "warmup": warm,
         "ms_per_step": round(ms_step, 5),
         "higher_is_better": True,
@@ -350,31 +379,37 @@ def run_ours(args, world, rank, local):
             "parallelism": f"replicas x{n}" if n > 1 else "1 GPU",
             "l2": f"rotating {R} weight copies ({R * step_bytes / 1e6:.0f} MB, > 3x L2): every step L2-cold",
             "seed": synth.BASE_SEED,
-            "timing": "K steps replayed from one CUDA graph, CUDA events on the replay stream; "
-                      "body_only/head_only (roofline): K launches of that kernel alone, replayed the same way",
+            "body_path": "48 weights in the streaming layout (repacked once at load, same bytes), "
+                         "w4r_matmul_grouped; head: i8_head_logits",
+            "timing": "a CUDA graph of K steps replayed back to back for about --seconds, CUDA events on the "
+                      "replay stream; body_only/head_only (roofline): K launches of that kernel alone per graph, "
+                      "replayed the same way",
         },
         "tokens_per_s": round(n * 1e3 / ms_step, 1),
         "body_only": {"ms": round(body_avg, 5), "GB_per_s": round(achieved, 1),
-                      "tokens_per_s": round(1e3 / body_avg, 1)},
+                      "tokens_per_s": round(1e3 / body_avg, 1), "launches_timed": K * n_body},
+        "body_page_format": {"ms": round(page_avg, 5),
+                             "GB_per_s": round(body_bytes() / (page_avg * 1e-3) / 1e9, 1),
+                             "kernel": "w4_gemv_kernel<1> (split-K GEMV on the page-format buffers)"},
         "head_only": {"ms": round(head_avg, 5),
                       "GB_per_s": round(head_bytes() / (head_avg * 1e-3) / 1e9, 1),
                       "frac_of_hbm": round(head_bytes() / (head_avg * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                       "traffic": profiled_traffic("i8_rows_gpt2_head_m1.md")},
         "frac_of_hbm_step": round(value / n / peaks["hbm_gbs"], 4),
         "roofline": {
-            "kernel": "w4_gemv_kernel<1> (grouped 48-weight launch)",
+            "kernel": "w4r_gemv_m1_kernel (48 repacked weights, one grouped launch)",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"],
             "peak_source": f"{peaks['_source']} hbm_gbs (copy, burst)",
             "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": profiled_traffic("w4_gemv_gpt2_m1.md"),
-            "traffic_source": "profiles/w4_gemv_gpt2_m1.md (ncu dram__bytes_read.sum + dram__bytes_write.sum, "
+            "traffic": profiled_traffic("w4r_gemv_gpt2_m1.md"),
+            "traffic_source": "profiles/w4r_gemv_gpt2_m1.md (ncu dram__bytes_read.sum + dram__bytes_write.sum, "
                               "one launch; null when the kernel source changed since)",
         },
         "e2e": e2e,
-        "gpu_launches": 2 * K,  # in the step graph's timed replay
+        "gpu_launches": 2 * steps_timed,  # body + head per step in the timed replays
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -647,6 +682,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--seconds", type=float, default=1.0,
+                    help="device seconds of the timed step replays (the body and head alone get half each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
                     help="decode: the GPT-2 decode step (the headline); prefill: the 3.8B-shaped stack at M=2048")

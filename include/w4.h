@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define W4_ABI_VERSION 2
+#define W4_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define W4_API __attribute__((visibility("default")))
@@ -197,6 +197,75 @@ W4_API w4_status w4_matmul_noalloc(const float* x, int64_t ldx, const uint8_t* q
 W4_API size_t w4_matmul_grouped_workspace_size(const w4_desc* descs, int32_t count);
 W4_API w4_status w4_matmul_grouped(const w4_desc* descs, int32_t count, void* workspace,
                             size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ streaming layout (decode) */
+
+/* The streaming layout of one W4 weight: the same 32-bit words as the three
+ * page-format buffers above (nibble words of 8 consecutive columns of one
+ * row, fp32 scales, zero-point words of 8 columns; "ONNX export, quantization
+ * and the browser runtime", section "Quantization (train/quantize.py)",
+ * step 2), reordered once at load time into the order in which the decode
+ * GEMV streams them, so that each of its warps reads one contiguous run of
+ * bytes. Nothing is added, rounded or dropped: w4_repack_restore gives back
+ * the page-format buffers bit for bit.
+ *
+ * Layout, K % 32 == 0, N % 8 == 0, nb = K / 32, gs = 32 / gcd(nb, 32),
+ * A = gs * nb / 32: groups of 8 gs columns (all K rows) in column order, each
+ * group A rounds of 5248 bytes. In round r of group G, lane l (0..31) owns
+ * strip s = l % gs (columns c0 = 8 (G gs + s) .. c0 + 7) and block
+ * b = l / gs + r * (32 / gs); its bytes are
+ *   nibble word of row 32 b + 4 c + j (c, j in 0..7, 0..3) at c*512 + l*16 + j*4
+ *     (the page's 4-byte word of row 32 b + 4 c + j, columns c0..c0+7),
+ *   scale of column c0 + i (i in 0..7) at 4096 + (i/4)*512 + l*16 + (i%4)*4,
+ *   zero-point word of block b, columns c0..c0+7, at 5120 + l*4.
+ * Strips at or past N (N not a multiple of 8 gs) hold zeros.
+ * w4_repacked_bytes() is the buffer size: K*N/2 + (K/32)*N*4 + (K/32)*N/2
+ * bytes (the page-format total) when N is a multiple of 8 gs, a little more
+ * otherwise; 0 for a shape the layout does not take. */
+W4_API size_t w4_repacked_bytes(int64_t K, int64_t N);
+
+/* Page format -> streaming layout, on the GPU. qw / scales / zp as for
+ * w4_matmul, wr: w4_repacked_bytes(K, N) bytes of device memory; all four
+ * 16-byte aligned. Asynchronous, stream-ordered. W4_ERR_SHAPE unless
+ * K % 32 == 0, N % 8 == 0 and 0 < K, N <= 2^30. */
+W4_API w4_status w4_repack(const uint8_t* qw, const float* scales, const uint8_t* zp, int64_t K, int64_t N,
+                           void* wr, void* stream);
+
+/* Streaming layout -> page format (the exact inverse of w4_repack). */
+W4_API w4_status w4_repack_restore(const void* wr, int64_t K, int64_t N, uint8_t* qw, float* scales, uint8_t* zp,
+                                   void* stream);
+
+/* One decode matmul on a repacked weight: y[1, N] = act(x[1, K] . W + bias)
+ * + residual, the fields and the epilogue as in w4_desc (ldx / ldy / ldr are
+ * not used: one row). Requires M == 1 (W4_ERR_SHAPE otherwise), K % 32 == 0,
+ * K <= 32768, N % 8 == 0, x and wr 16-byte aligned, y / bias / residual
+ * 4-byte aligned. No workspace: every output column is summed inside one
+ * warp. reserved must be 0. */
+typedef struct w4r_desc {
+  const float* x;
+  int64_t ldx;
+  const void* wr;
+  float* y;
+  int64_t ldy;
+  int64_t M;
+  int64_t K;
+  int64_t N;
+  const float* bias;
+  const float* residual;
+  int64_t ldr;
+  int32_t act;
+  int32_t reserved;
+} w4r_desc;
+
+/* Many independent decode matmuls on repacked weights in as few launches as
+ * possible (64 per launch). `descs` is a HOST array read during the call
+ * only; outputs must not overlap each other or any input. The launch lets the
+ * next launch on the stream begin streaming its weights while this one
+ * finishes (programmatic dependent launch); x is read and y written only
+ * after the previous work on the stream has completed, so the usual stream
+ * order holds for every input and output. */
+W4_API w4_status w4r_matmul_grouped(const w4r_desc* descs, int32_t count, void* stream);
+W4_API w4_status w4r_matmul(const w4r_desc* d, void* stream);
 
 /* ------------------------------------------------------------------ head */
 

@@ -9,6 +9,8 @@ Operations (see include/w4.h for layouts and error behaviour):
   w4_matmul(x, qw, scales, zp, K, N)        y = x . W, W 4-bit blocked
       (..., bias=, residual=, act=)         y = act(x . W + bias) + residual, fused
   w4_matmul_grouped([...])                  many independent ones, one launch
+  w4_repack(qw, scales, zp, K, N)           the weight in the streaming layout (once, at load)
+  w4r_matmul(x, wr, K, N) / _grouped        decode (M = 1) on repacked weights
   i8_head_logits(h, table, scales, K, V)    last-position logits, int8 head
   w4_quantize(w, block, scale_type)         the dq4 quantiser (GPU)
   i8_quantize_head(w)                       the embedding_int8 quantiser (GPU)
@@ -23,7 +25,7 @@ from typing import Sequence
 import numpy as np
 
 from . import _lib
-from ._lib import ACTS, GROUP_MAX, PATHS, STATUS, W4Desc, W4LibraryMissing  # noqa: F401
+from ._lib import ACTS, GROUP_MAX, PATHS, STATUS, W4Desc, W4LibraryMissing, W4RDesc  # noqa: F401
 
 
 class W4Error(RuntimeError):
@@ -169,6 +171,71 @@ def w4_matmul_grouped(items: Sequence[dict] | None = None, descs=None, ws=None, 
     st = lib().w4_matmul_grouped(descs, len(descs), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                  _stream_handle(stream))
     _check(st, "w4_matmul_grouped")
+
+
+# ---------------------------------------------------------------- streaming layout (decode)
+
+def w4_repacked_bytes(K: int, N: int) -> int:
+    return int(lib().w4_repacked_bytes(K, N))
+
+
+def w4_repack(qw, scales, zp, K: int, N: int, out=None, stream=None):
+    """The weight (page format: packed nibbles, fp32 scales, packed zero
+    points) in the streaming layout the decode GEMV reads: a uint8 device
+    tensor of w4_repacked_bytes(K, N) bytes holding the same words, reordered."""
+    torch = _torch()
+    nbytes = w4_repacked_bytes(K, N)
+    if nbytes == 0:
+        raise ValueError(f"the streaming layout does not take K={K}, N={N} (K % 32 == 0, N % 8 == 0)")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=qw.device)
+    st = lib().w4_repack(_ptr(qw), _ptr(scales), _ptr(zp), K, N, _ptr(out), _stream_handle(stream))
+    _check(st, "w4_repack")
+    return out
+
+
+def w4_repack_restore(wr, K: int, N: int, stream=None):
+    """The page-format buffers (qw, scales, zp) of a repacked weight."""
+    torch = _torch()
+    nb = K // 32
+    qw = torch.empty(K * N // 2, dtype=torch.uint8, device=wr.device)
+    sc = torch.empty((nb, N), dtype=torch.float32, device=wr.device)
+    zp = torch.empty(nb * N // 2, dtype=torch.uint8, device=wr.device)
+    st = lib().w4_repack_restore(_ptr(wr), K, N, _ptr(qw), _ptr(sc), _ptr(zp), _stream_handle(stream))
+    _check(st, "w4_repack_restore")
+    return qw, sc, zp
+
+
+def make_rdescs(items: Sequence[dict]):
+    """ctypes w4r_desc array for w4r_matmul_grouped; each item holds the
+    tensors x ([1, K] or [K]), wr (repacked), y and the ints K, N, and
+    optionally "bias", "residual" and "act"."""
+    arr = (W4RDesc * len(items))()
+    for i, it in enumerate(items):
+        x, y = it["x"], it["y"]
+        K, N = int(it["K"]), int(it["N"])
+        M = x.shape[0] if x.dim() == 2 else 1
+        b, r, ldr, a = _epilogue(it, N)
+        arr[i] = W4RDesc(_ptr(x), K, _ptr(it["wr"]), _ptr(y), N, M, K, N, b, r, ldr, a, 0)
+    return arr
+
+
+def w4r_matmul_grouped(items: Sequence[dict] | None = None, descs=None, stream=None):
+    """All decode matmuls of `items` (or a prepared w4r_desc array)."""
+    if descs is None:
+        descs = make_rdescs(items)
+    st = lib().w4r_matmul_grouped(descs, len(descs), _stream_handle(stream))
+    _check(st, "w4r_matmul_grouped")
+
+
+def w4r_matmul(x, wr, K: int, N: int, y=None, stream=None, bias=None, residual=None, act: str = "none"):
+    """y[1, N] = act(x[1, K] . W + bias) + residual with W repacked (w4_repack)."""
+    torch = _torch()
+    if y is None:
+        y = torch.empty((1, N), dtype=torch.float32, device=x.device)
+    item = {"x": x, "wr": wr, "y": y, "K": K, "N": N, "bias": bias, "residual": residual, "act": act}
+    w4r_matmul_grouped(descs=make_rdescs([item]), stream=stream)
+    return y
 
 
 # ---------------------------------------------------------------- head

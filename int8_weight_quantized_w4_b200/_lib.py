@@ -27,7 +27,7 @@ W4_OK, W4_ERR_NULL, W4_ERR_SHAPE, W4_ERR_ALIGN, W4_ERR_DEVICE, W4_ERR_CUDA, W4_E
     W4_ERR_VALUE = range(9)
 PATHS = {"auto": 0, "gemv": 1, "generic": 2, "tc": 3}
 ACTS = {"none": 0, "gelu_tanh": 1, "gelu_erf": 2}
-ABI_VERSION = 2
+ABI_VERSION = 3
 GROUP_MAX = 48
 
 
@@ -38,6 +38,25 @@ class W4Desc(C.Structure):
         ("qw", C.c_void_p),
         ("scales", C.c_void_p),
         ("zp", C.c_void_p),
+        ("y", C.c_void_p),
+        ("ldy", C.c_int64),
+        ("M", C.c_int64),
+        ("K", C.c_int64),
+        ("N", C.c_int64),
+        ("bias", C.c_void_p),
+        ("residual", C.c_void_p),
+        ("ldr", C.c_int64),
+        ("act", C.c_int32),
+        ("reserved", C.c_int32),
+    ]
+
+
+class W4RDesc(C.Structure):
+    """w4r_desc: one decode matmul on a weight in the streaming layout."""
+    _fields_ = [
+        ("x", C.c_void_p),
+        ("ldx", C.c_int64),
+        ("wr", C.c_void_p),
         ("y", C.c_void_p),
         ("ldy", C.c_int64),
         ("M", C.c_int64),
@@ -63,6 +82,12 @@ SIGNATURES = {
     "w4_matmul_desc": (C.c_int, [C.POINTER(W4Desc), C.c_void_p, C.c_size_t, C.c_int, C.c_void_p]),
     "w4_matmul_grouped_workspace_size": (C.c_size_t, [C.POINTER(W4Desc), C.c_int32]),
     "w4_matmul_grouped": (C.c_int, [C.POINTER(W4Desc), C.c_int32, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "w4_repacked_bytes": (C.c_size_t, [C.c_int64, C.c_int64]),
+    "w4_repack": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),
+    "w4_repack_restore": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p,
+                                    C.c_void_p]),
+    "w4r_matmul": (C.c_int, [C.POINTER(W4RDesc), C.c_void_p]),
+    "w4r_matmul_grouped": (C.c_int, [C.POINTER(W4RDesc), C.c_int32, C.c_void_p]),
     "i8_head_workspace_size": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int64]),
     "i8_head_argmax_workspace_size": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int64]),
     "i8_head_argmax": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_int64,

@@ -1,0 +1,561 @@
+// w4r: the streaming layout of a W4 weight, and the decode GEMV (M = 1) that
+// reads it.
+//
+// The weight format is the one of "ONNX export, quantization and the browser
+// runtime", section "Quantization (train/quantize.py)", step 2 (dq4): blocks
+// of 32 along K, one fp32 scale and one uint4 zero point per (block,
+// column), w = (q - zp) * scale. The streaming layout holds exactly the same
+// 32-bit words as the three page-format buffers (nibble words of 8
+// consecutive columns of one row, fp32 scales, zero-point words of 8
+// columns), only in another order: the order in which one warp of the GEMV
+// consumes them. Repacking is a permutation of words, done once when the
+// weights are loaded; the GEMV then streams each warp's share of the weight as
+// one contiguous run of bytes, so every copy is a plain bulk copy with no
+// tensor map, no split along K and no scratch memory.
+//
+// Layout (K % 32 == 0, N % 8 == 0; nb = K / 32):
+//   gs = 32 / gcd(nb, 32) strips of 8 columns form a group (8 * gs columns,
+//   all K rows); A = gs * nb / 32 rounds make a group; a round is 5248 bytes,
+//   one 164-byte "atom" (8 columns x 32 rows, one block) for each of 32 lanes:
+//     lane l: strip s = l % gs, phase p = l / gs, block b = p + r * (32 / gs)
+//     [0, 4096)     nibble words: word j of 16-byte chunk c of lane l at
+//                   c * 512 + l * 16 + j * 4 is row 32 b + 4 c + j, columns
+//                   8 (G gs + s) .. +7 of the [K, N] nibble tensor (the
+//                   page's aligned 4-byte word: nibble i = column +i)
+//     [4096, 5120)  scales: float i of lane l at 4096 + (i / 4) * 512 + l * 16
+//                   + (i % 4) * 4 is scale[b][8 (G gs + s) + i]
+//     [5120, 5248)  zero-point words: lane l at 5120 + l * 4 (nibble i = the
+//                   zero point of column +i in block b)
+//   Groups follow each other in column order; strips past N (when N is not a
+//   multiple of 8 gs) are zero in the repacked buffer and never written.
+//
+// GEMV design (sm_100a, M = 1):
+//  * A CTA is 4 warps; each warp owns one group (8 gs columns, all of K), so
+//    every output column is summed by one warp with no partial sums in
+//    memory. For the GPT-2 and 3.8B shapes every group is 96 atoms (15.7 KB)
+//    or, for K = 8192, 256 atoms.
+//  * Each warp streams its group through a ring of 3 stages of one round,
+//    with one bulk copy per round issued by its lane 0 (no multicast); for
+//    A <= 3 the whole group is requested at the CTA's first instruction.
+//  * The CTA stages x in shared memory as [row quad c][block b][4 floats] so
+//    that lanes reading different blocks hit different banks.
+//  * The launch lets the next launch in the stream start early (programmatic
+//    dependent launch): a CTA requests its weight bytes before it waits for
+//    the previous launch to finish, and reads x / writes y only after that
+//    wait. The weights are constants of the model; x and y may belong to the
+//    previous launch.
+//  * Dequantisation: one LOP3 per weight builds the float 2^23 + q*16^j
+//    exactly (nibble j of a half-word); rows k and k+1 are taken together, so
+//    one FADD2 subtracts the zero point's float from both (exact) and one
+//    FFMA2 accumulates with (x_k, x_k+1). The scale (times 16^-j) is applied
+//    once per block and column: y += s * sum_k x_k (q_k - zp).
+//  * The 32 / gs lanes of a strip are added by a butterfly of shuffles; the
+//    lane with phase 0 writes 8 columns through the fused epilogue.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "w4_device.cuh"
+#include "w4_internal.h"
+
+namespace {
+
+using namespace w4dev;
+
+constexpr int ROUND_BYTES = 5248;
+constexpr int NIB_BYTES = 4096;
+constexpr int SC_BYTES = 1024;
+constexpr int ROUND_WORDS = ROUND_BYTES / 4;  // 1312
+constexpr int RW = 4;                         // warps per CTA
+constexpr int NST = 3;                        // stages per warp
+constexpr int RCAP = 64;                      // matrices per launch
+constexpr int STAGE_SMEM = RW * NST * ROUND_BYTES;
+
+struct RMat {
+  const uint8_t* wr;
+  const float* x;
+  float* y;
+  const float* bias;
+  const float* res;
+  int64_t ldr;
+  int32_t K;
+  int32_t N;
+  int32_t cta0;     // first CTA of this matrix in the launch
+  int32_t ngroups;  // groups of 8 gs columns
+  int32_t act;
+  int32_t gsl;      // log2(gs)
+};
+
+struct RParams {
+  RMat m[RCAP];
+  int32_t count;
+  int32_t x_floats;  // shared-memory floats reserved for x
+  ErrorWord* err;
+  uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// One atom: 8 columns x 32 rows for this lane, accumulated into acc[0..7].
+// st: the stage; xb: x of the atom's block in the [c][b][4] layout, c-th
+// quad at xb + c * xq floats.
+__device__ __forceinline__ void atom_m1(const uint8_t* st, int lane, const float* xb, int xq, uint32_t kMagic,
+                                        float (&acc)[8]) {
+  const uint32_t zw = *reinterpret_cast<const uint32_t*>(st + NIB_BYTES + SC_BYTES + lane * 4);
+  float2 nz[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float z = -magic_nib(i < 4 ? zw : (zw >> 16), i & 3);
+    nz[i] = make_float2(z, z);
+  }
+  float2 P[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) P[i] = make_float2(0.f, 0.f);
+#pragma unroll 2
+  for (int c = 0; c < 8; ++c) {
+    const uint4 wv = *reinterpret_cast<const uint4*>(st + c * 512 + lane * 16);
+    const float4 x4 = *reinterpret_cast<const float4*>(xb + c * xq);
+    const float2 xa = make_float2(x4.x, x4.y);
+    const float2 xb2 = make_float2(x4.z, x4.w);
+    const uint32_t wl[4] = {wv.x, wv.y, wv.z, wv.w};
+    uint32_t wh[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) wh[t] = __umulhi(wl[t], 65536u);  // wl >> 16 on the FMA pipe
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int sl = i & 3;
+      const float2 m01 = make_float2(magic_nib_r(i < 4 ? wl[0] : wh[0], kMagic, sl),
+                                     magic_nib_r(i < 4 ? wl[1] : wh[1], kMagic, sl));
+      const float2 m23 = make_float2(magic_nib_r(i < 4 ? wl[2] : wh[2], kMagic, sl),
+                                     magic_nib_r(i < 4 ? wl[3] : wh[3], kMagic, sl));
+      P[i] = __ffma2_rn(xa, __fadd2_rn(m01, nz[i]), P[i]);
+      P[i] = __ffma2_rn(xb2, __fadd2_rn(m23, nz[i]), P[i]);
+    }
+  }
+  const float4 s0 = *reinterpret_cast<const float4*>(st + NIB_BYTES + lane * 16);
+  const float4 s1 = *reinterpret_cast<const float4*>(st + NIB_BYTES + 512 + lane * 16);
+  const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = fmaf(P[i].x + P[i].y, sv[i] * inv_slot_scale(i & 3), acc[i]);
+}
+
+__global__ void __launch_bounds__(RW * 32, 3) w4r_gemv_m1_kernel(const __grid_constant__ RParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // matrix of this CTA: the last one whose first CTA is at or before it
+  int g = 0;
+  {
+    int lo = 0, hi = p.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.m[mid].cta0 <= static_cast<int>(blockIdx.x)) lo = mid;
+      else hi = mid - 1;
+    }
+    g = lo;
+  }
+  const RMat& m = p.m[g];
+  const int K = m.K;
+  const int nb = K >> 5;
+  const int gsl = m.gsl;
+  const int A = (nb << gsl) >> 5;  // rounds of a group
+  const int group = (static_cast<int>(blockIdx.x) - m.cta0) * RW + warp;
+  const bool active = group < m.ngroups;
+
+  uint8_t* stg = smem + warp * (NST * ROUND_BYTES);
+  float* xs = reinterpret_cast<float*>(smem + STAGE_SMEM);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + STAGE_SMEM + p.x_floats * 4) + warp * NST;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + STAGE_SMEM + p.x_floats * 4 + RW * NST * 8) + warp;
+  const uint8_t* src = m.wr + static_cast<int64_t>(group) * A * ROUND_BYTES;
+
+  // ---- weights first: they do not depend on the previous launch
+  int issued = 0;  // rounds requested (lane 0)
+  if (active && lane == 0) {
+    for (int s = 0; s < NST; ++s) mbar_init(&bar[s], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    const int n0 = min(A, NST);
+    for (int r = 0; r < n0; ++r) {
+      mbar_arrive_expect_tx(&bar[r], ROUND_BYTES);
+      bulk_g2s(stg + r * ROUND_BYTES, src + static_cast<int64_t>(r) * ROUND_BYTES, ROUND_BYTES, &bar[r]);
+    }
+    issued = n0;
+  }
+  __syncwarp();
+  pdl_launch_dependents();
+  pdl_wait();  // x and y may be the previous launch's
+
+  // ---- x of this CTA's matrix into shared memory, [quad c][block b][4]
+  for (int i = threadIdx.x; i < (K >> 2); i += RW * 32) {
+    const int b = i >> 3, c = i & 7;
+    cp_async_16(xs + (c * nb + b) * 4, m.x + 4 * i, 16);
+  }
+  cp_async_commit();
+  cp_async_wait_group<0>();
+  __syncthreads();
+  if (!active) return;
+
+  uint32_t kMagic;  // 0x4B000000 (the bits of 2^23) held in a register
+  asm("mov.b32 %0, 0x4B000000;" : "=r"(kMagic));
+  const int gs = 1 << gsl;
+  const int strip = lane & (gs - 1);
+  const int phase = lane >> gsl;
+  const int pstride = 32 >> gsl;
+  const int xq = nb * 4;  // floats between row quads of x
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+
+  bool ok = true;
+  int s = 0;
+  uint32_t par = 0;
+#pragma unroll 1
+  for (int r = 0; r < A; ++r) {
+    ok = mbar_wait_bounded(&bar[s], par, p.timeout_ns, abort_flag, p.err, K_GEMVR, 1);
+    if (__any_sync(0xffffffffu, !ok)) {
+      ok = false;
+      break;
+    }
+    const int b = phase + r * pstride;
+    atom_m1(stg + s * ROUND_BYTES, lane, xs + b * 4, xq, kMagic, acc);
+    __syncwarp();
+    if (lane == 0 && issued < A) {  // refill this stage with the round NST ahead
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&bar[s], ROUND_BYTES);
+      bulk_g2s(stg + s * ROUND_BYTES, src + static_cast<int64_t>(issued) * ROUND_BYTES, ROUND_BYTES, &bar[s]);
+      ++issued;
+    }
+    if (++s == NST) {
+      s = 0;
+      par ^= 1u;
+    }
+  }
+
+  if (!ok) {
+    // copies still in flight must land before the CTA exits: wait (bounded)
+    // for the last fill of every stage
+    if (lane == 0)
+      for (int st = 0; st < NST; ++st) {
+        const int fills = issued > st ? (issued - st + NST - 1) / NST : 0;
+        if (fills > 0) mbar_wait_bounded(&bar[st], (fills - 1) & 1, p.timeout_ns, nullptr, p.err, K_GEMVR, 2);
+      }
+    return;
+  }
+
+  // ---- the lanes of a strip: butterfly over the phase bits
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    for (int off = gs; off < 32; off <<= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+  if (phase != 0) return;
+  const int col = ((group << gsl) + strip) * 8;
+  if (col >= m.N) return;
+  float* yp = m.y + col;
+  const Epi epi{m.bias, m.res, m.ldr, m.act, 0};
+  float v[8];
+  if (epi_active(epi)) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = epi_apply(acc[i], epi, 0, col + i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = acc[i];
+  }
+  if ((reinterpret_cast<uintptr_t>(yp) & 15) == 0) {
+    reinterpret_cast<float4*>(yp)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(yp)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) yp[i] = v[i];
+  }
+}
+
+// ---------------------------------------------------------------- repacking
+
+struct RepackGeom {
+  int32_t nb, gsl, A, ngroups;
+  int64_t words;  // 32-bit words of the repacked buffer
+};
+
+// Where word o of the repacked buffer comes from: kind 0 nibble word, 1
+// scale, 2 zero-point word; src = its index in that page-format array as
+// 32-bit words; false for a padding word (a strip past N).
+__device__ __forceinline__ bool repack_source(int64_t o, const RepackGeom& g, int64_t N, int* kind, int64_t* src) {
+  const int64_t round_id = o / ROUND_WORDS;
+  const int w = static_cast<int>(o - round_id * ROUND_WORDS);
+  const int64_t group = round_id / g.A;
+  const int r = static_cast<int>(round_id - group * g.A);
+  int lane, row = 0, i = 0;
+  if (w < 1024) {
+    const int c = w >> 7;
+    lane = (w >> 2) & 31;
+    row = 4 * c + (w & 3);
+    *kind = 0;
+  } else if (w < 1280) {
+    const int v = w - 1024;
+    lane = (v >> 2) & 31;
+    i = (v >> 7) * 4 + (v & 3);
+    *kind = 1;
+  } else {
+    lane = w - 1280;
+    *kind = 2;
+  }
+  const int gs = 1 << g.gsl;
+  const int strip = lane & (gs - 1);
+  const int phase = lane >> g.gsl;
+  const int64_t b = phase + static_cast<int64_t>(r) * (32 >> g.gsl);
+  const int64_t col = (group * gs + strip) * 8;
+  if (col >= N) return false;
+  if (*kind == 0) *src = ((b * 32 + row) * N + col) >> 3;
+  else if (*kind == 1) *src = b * N + col + i;
+  else *src = (b * N + col) >> 3;
+  return true;
+}
+
+__global__ void w4r_repack_kernel(const uint32_t* __restrict__ qw, const uint32_t* __restrict__ sc,
+                                  const uint32_t* __restrict__ zp, int64_t N, RepackGeom g, uint32_t* __restrict__ out) {
+  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < g.words;
+       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int kind;
+    int64_t s;
+    uint32_t v = 0;
+    if (repack_source(o, g, N, &kind, &s)) v = kind == 0 ? qw[s] : (kind == 1 ? sc[s] : zp[s]);
+    out[o] = v;
+  }
+}
+
+__global__ void w4r_restore_kernel(const uint32_t* __restrict__ in, int64_t N, RepackGeom g, uint32_t* __restrict__ qw,
+                                   uint32_t* __restrict__ sc, uint32_t* __restrict__ zp) {
+  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < g.words;
+       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int kind;
+    int64_t s;
+    if (repack_source(o, g, N, &kind, &s)) {
+      if (kind == 0) qw[s] = in[o];
+      else if (kind == 1) sc[s] = in[o];
+      else zp[s] = in[o];
+    }
+  }
+}
+
+int gcd32(int a) {
+  int b = 32;
+  while (b != 0) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+
+bool geom_of(int64_t K, int64_t N, RepackGeom* g) {
+  if (K <= 0 || N <= 0 || K % 32 != 0 || N % 8 != 0 || K > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return false;
+  g->nb = static_cast<int32_t>(K / 32);
+  const int gs = 32 / gcd32(g->nb);
+  g->gsl = __builtin_ctz(gs);
+  g->A = g->nb / gcd32(g->nb);
+  g->ngroups = static_cast<int32_t>((N + 8 * gs - 1) / (8 * gs));
+  g->words = static_cast<int64_t>(g->ngroups) * g->A * ROUND_WORDS;
+  return true;
+}
+
+bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+w4_status launch_repack_like(bool restore, const uint8_t* qw, const float* sc, const uint8_t* zp, const void* wr,
+                             int64_t K, int64_t N, uint8_t* qw_out, float* sc_out, uint8_t* zp_out, void* wr_out,
+                             cudaStream_t st) {
+  using namespace w4host;
+  RepackGeom g;
+  if (!geom_of(K, N, &g))
+    return fail(W4_ERR_SHAPE, "streaming layout needs K %% 32 == 0, N %% 8 == 0, 0 < K, N <= 2^30 (K=%lld N=%lld)",
+                static_cast<long long>(K), static_cast<long long>(N));
+  const DeviceInfo* di = nullptr;
+  w4_status rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  const int64_t blocks = std::min<int64_t>((g.words + 255) / 256, static_cast<int64_t>(di->sms) * 32);
+  if (!restore) {
+    w4r_repack_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        reinterpret_cast<const uint32_t*>(qw), reinterpret_cast<const uint32_t*>(sc),
+        reinterpret_cast<const uint32_t*>(zp), N, g, static_cast<uint32_t*>(wr_out));
+  } else {
+    w4r_restore_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint32_t*>(wr), N, g, reinterpret_cast<uint32_t*>(qw_out), reinterpret_cast<uint32_t*>(sc_out),
+        reinterpret_cast<uint32_t*>(zp_out));
+  }
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W4_OK : cuda_fail(e, restore ? "launch w4r_restore" : "launch w4r_repack");
+}
+
+// ---------------------------------------------------------------- GEMV launch
+
+w4_status check_rdesc(const w4r_desc& d, RepackGeom* g) {
+  using namespace w4host;
+  if (d.M < 0 || d.K < 0 || d.N < 0) return fail(W4_ERR_SHAPE, "negative size");
+  if (d.act < W4_ACT_NONE || d.act > W4_ACT_GELU_ERF) return fail(W4_ERR_VALUE, "unknown activation %d", int(d.act));
+  if (d.reserved != 0) return fail(W4_ERR_VALUE, "reserved field must be 0");
+  if (d.M == 0 || d.N == 0) return W4_OK;
+  if (d.N % 8 != 0) return fail(W4_ERR_SHAPE, "streaming layout needs N %% 8 == 0 (N=%lld)", (long long)d.N);
+  if (d.K % 32 != 0) return fail(W4_ERR_SHAPE, "K=%lld is not a multiple of 32", (long long)d.K);
+  if (d.M != 1) return fail(W4_ERR_SHAPE, "the streaming-layout GEMV takes M = 1 (M=%lld)", (long long)d.M);
+  if (d.y == nullptr) return fail(W4_ERR_NULL, "y is NULL");
+  if (!aligned_to(d.y, 4)) return fail(W4_ERR_ALIGN, "y must be 4-byte aligned");
+  if (d.bias != nullptr && !aligned_to(d.bias, 4)) return fail(W4_ERR_ALIGN, "bias must be 4-byte aligned");
+  if (d.residual != nullptr && !aligned_to(d.residual, 4))
+    return fail(W4_ERR_ALIGN, "residual must be 4-byte aligned");
+  if (d.K == 0) return W4_OK;
+  if (d.x == nullptr || d.wr == nullptr) return fail(W4_ERR_NULL, "x and wr must not be NULL");
+  if (!aligned_to(d.x, 16)) return fail(W4_ERR_ALIGN, "the streaming-layout GEMV needs x 16-byte aligned");
+  if (!aligned_to(d.wr, 16)) return fail(W4_ERR_ALIGN, "the repacked weight must be 16-byte aligned");
+  if (d.K > 32768) return fail(W4_ERR_SHAPE, "the streaming-layout GEMV takes K <= 32768 (K=%lld)", (long long)d.K);
+  geom_of(d.K, d.N, g);
+  return W4_OK;
+}
+
+int rsmem_bytes(int x_floats) { return STAGE_SMEM + x_floats * 4 + RW * NST * 8 + RW * 4; }
+
+w4_status launch_rgroup(const w4r_desc* d, const RepackGeom* geo, int count, cudaStream_t st,
+                        const w4host::DeviceInfo& di) {
+  using namespace w4host;
+  RParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  int cta = 0;
+  int xf = 0;
+  for (int i = 0; i < count; ++i) {
+    RMat& m = prm.m[i];
+    const RepackGeom& g = geo[i];
+    m.wr = static_cast<const uint8_t*>(d[i].wr);
+    m.x = d[i].x;
+    m.y = d[i].y;
+    m.bias = d[i].bias;
+    m.res = d[i].residual;
+    m.ldr = d[i].ldr;
+    m.K = static_cast<int32_t>(d[i].K);
+    m.N = static_cast<int32_t>(d[i].N);
+    m.cta0 = cta;
+    m.ngroups = g.ngroups;
+    m.act = d[i].act;
+    m.gsl = g.gsl;
+    cta += (g.ngroups + RW - 1) / RW;
+    xf = std::max(xf, m.K);
+  }
+  prm.count = count;
+  prm.x_floats = xf;
+  prm.err = di.err;
+  prm.timeout_ns = wait_timeout_ns();
+  const int smem = rsmem_bytes(xf);
+  static int configured[64] = {};
+  if (di.dev < 64 && configured[di.dev] < smem) {
+    const cudaError_t e = cudaFuncSetAttribute(w4r_gemv_m1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               rsmem_bytes(32768));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(w4r_gemv)");
+    configured[di.dev] = rsmem_bytes(32768);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(cta));
+  cfg.blockDim = dim3(RW * 32);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, w4r_gemv_m1_kernel, prm);
+  return e == cudaSuccess ? W4_OK : cuda_fail(e, "launch w4r_gemv");
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t w4_repacked_bytes(int64_t K, int64_t N) {
+  RepackGeom g;
+  if (!geom_of(K, N, &g)) return 0;
+  return static_cast<size_t>(g.words) * 4;
+}
+
+w4_status w4_repack(const uint8_t* qw, const float* scales, const uint8_t* zp, int64_t K, int64_t N, void* wr,
+                    void* stream) {
+  using namespace w4host;
+  if (qw == nullptr || scales == nullptr || zp == nullptr || wr == nullptr)
+    return fail(W4_ERR_NULL, "qw, scales, zp and wr must not be NULL");
+  if (!aligned_to(qw, 16) || !aligned_to(scales, 16) || !aligned_to(zp, 16) || !aligned_to(wr, 16))
+    return fail(W4_ERR_ALIGN, "qw, scales, zp and wr must be 16-byte aligned");
+  return launch_repack_like(false, qw, scales, zp, nullptr, K, N, nullptr, nullptr, nullptr, wr,
+                            static_cast<cudaStream_t>(stream));
+}
+
+w4_status w4_repack_restore(const void* wr, int64_t K, int64_t N, uint8_t* qw, float* scales, uint8_t* zp,
+                            void* stream) {
+  using namespace w4host;
+  if (qw == nullptr || scales == nullptr || zp == nullptr || wr == nullptr)
+    return fail(W4_ERR_NULL, "qw, scales, zp and wr must not be NULL");
+  if (!aligned_to(qw, 16) || !aligned_to(scales, 16) || !aligned_to(zp, 16) || !aligned_to(wr, 16))
+    return fail(W4_ERR_ALIGN, "qw, scales, zp and wr must be 16-byte aligned");
+  return launch_repack_like(true, nullptr, nullptr, nullptr, wr, K, N, qw, scales, zp, nullptr,
+                            static_cast<cudaStream_t>(stream));
+}
+
+w4_status w4r_matmul_grouped(const w4r_desc* descs, int32_t count, void* stream) {
+  using namespace w4host;
+  if (count < 0) return fail(W4_ERR_SHAPE, "negative count");
+  if (count == 0) return W4_OK;
+  if (descs == nullptr) return fail(W4_ERR_NULL, "descs is NULL");
+  static thread_local RepackGeom geo[RCAP];
+  static thread_local w4r_desc run[RCAP];
+  int work = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    RepackGeom g;
+    const w4_status rc = check_rdesc(descs[i], &g);
+    if (rc != W4_OK) {
+      char why[256];
+      snprintf(why, sizeof(why), "%s", w4_last_error());
+      return fail(rc, "descriptor %d: %s", i, why);
+    }
+    if (descs[i].M != 0 && descs[i].N != 0) ++work;
+  }
+  if (work == 0) return W4_OK;
+  const DeviceInfo* di = nullptr;
+  w4_status rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int n = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    const w4r_desc& d = descs[i];
+    if (d.M == 0 || d.N == 0) continue;
+    if (d.K == 0) {
+      w4_desc z = {};
+      z.bias = d.bias;
+      z.residual = d.residual;
+      z.ldr = d.ldr;
+      z.act = d.act;
+      rc = launch_zero_fill(d.y, d.N, 1, d.N, st, &z);
+      if (rc != W4_OK) return rc;
+      continue;
+    }
+    geom_of(d.K, d.N, &geo[n]);
+    run[n++] = d;
+    if (n == RCAP) {
+      rc = launch_rgroup(run, geo, n, st, *di);
+      if (rc != W4_OK) return rc;
+      n = 0;
+    }
+  }
+  if (n > 0) rc = launch_rgroup(run, geo, n, st, *di);
+  return rc;
+}
+
+w4_status w4r_matmul(const w4r_desc* d, void* stream) {
+  if (d == nullptr) return w4host::fail(W4_ERR_NULL, "descriptor is NULL");
+  return w4r_matmul_grouped(d, 1, stream);
+}
+
+}  // extern "C"

@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol():
 def test_abi_version_and_status_strings():
     lib = _lib()
     from int8_weight_quantized_w4_b200 import _lib as L
-    assert lib.w4_abi_version() == L.ABI_VERSION == 2
+    assert lib.w4_abi_version() == L.ABI_VERSION == 3
     assert lib.w4_status_string(0) == b"W4_OK"
     assert lib.w4_status_string(6) == b"W4_ERR_TIMEOUT"
     assert lib.w4_status_string(99) == b"W4_ERR_UNKNOWN"
@@ -197,3 +197,64 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(L, "_lib", None)
     with pytest.raises(L.W4LibraryMissing):
         L.load()
+
+
+# ---------------------------------------------------------------- streaming layout
+
+def test_repacked_bytes_is_the_page_format_total():
+    lib = _lib()
+    import math
+    for K, N in [(768, 768), (768, 2304), (3072, 768), (8192, 3072), (32, 256), (96, 768)]:
+        nb = K // 32
+        gs = 32 // math.gcd(nb, 32)
+        assert N % (8 * gs) == 0
+        assert lib.w4_repacked_bytes(K, N) == K * N // 2 + nb * N * 4 + nb * N // 2
+    # a last group that is only partly filled is padded to whole strips of the group
+    assert lib.w4_repacked_bytes(768, 200) == 7 * 3 * 5248
+    for K, N in [(33, 64), (64, 60), (0, 64), (64, 0), (-32, 64)]:
+        assert lib.w4_repacked_bytes(K, N) == 0
+
+
+def _rdesc(**kw):
+    from int8_weight_quantized_w4_b200._lib import W4RDesc
+    a = dict(x=0x1000, ldx=64, wr=0x2000, y=0x5000, ldy=64, M=1, K=64, N=64, bias=0, residual=0, ldr=0, act=0,
+             reserved=0)
+    a.update(kw)
+    return W4RDesc(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(M=2), 2), (dict(N=60), 2), (dict(K=40), 2), (dict(K=65536), 2), (dict(M=-1), 2),
+    (dict(x=0x1004), 3), (dict(wr=0x2008), 3), (dict(y=0x5002), 3), (dict(bias=0x6002), 3),
+    (dict(x=0), 1), (dict(wr=0), 1), (dict(y=0), 1), (dict(act=5), 8), (dict(reserved=1), 8),
+])
+def test_w4r_argument_errors_before_any_launch(kw, status):
+    lib = _lib()
+    d = _rdesc(**kw)
+    assert lib.w4r_matmul(C.byref(d), None) == status
+    assert lib.w4_last_error()
+
+
+def test_w4r_noops_and_repack_shape_errors_need_no_device():
+    lib = _lib()
+    assert lib.w4r_matmul(C.byref(_rdesc(M=0)), None) == 0
+    assert lib.w4r_matmul(C.byref(_rdesc(N=0, x=0, wr=0)), None) == 0
+    assert lib.w4r_matmul(None, None) == 1
+    assert lib.w4r_matmul_grouped(None, 0, None) == 0
+    assert lib.w4_repack(0x1000, 0x2000, 0x3000, 64, 60, 0x4000, None) == 2
+    assert lib.w4_repack(0x1000, 0x2000, 0x3000, 40, 64, 0x4000, None) == 2
+    assert lib.w4_repack(0x1000, 0x2004, 0x3000, 64, 64, 0x4000, None) == 3
+    assert lib.w4_repack(0, 0x2000, 0x3000, 64, 64, 0x4000, None) == 1
+    assert lib.w4_repack_restore(0x4000, 64, 62, 0x1000, 0x2000, 0x3000, None) == 2
+
+
+def test_rdesc_layout_matches_the_c_struct(tmp_path):
+    from int8_weight_quantized_w4_b200._lib import W4RDesc
+    src = tmp_path / "rlayout.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "w4.h"\n'
+                   'int main(void) { printf("%zu %zu %zu %zu %zu\\n", sizeof(w4r_desc), offsetof(w4r_desc, wr), '
+                   'offsetof(w4r_desc, N), offsetof(w4r_desc, ldr), offsetof(w4r_desc, act)); return 0; }\n')
+    exe = tmp_path / "rlayout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert got == [C.sizeof(W4RDesc), W4RDesc.wr.offset, W4RDesc.N.offset, W4RDesc.ldr.offset, W4RDesc.act.offset]
