@@ -11,9 +11,11 @@
 //
 // The scratch is one file-scope __device__ array of W4_NOALLOC_SCRATCH_BYTES.
 // Every GPU that loads the library holds it until the process exits, and all
-// calls share it: each call first clears the part it will use (the split-K
-// counters must start at zero), and calls whose work overlaps on the GPU
-// (different streams, or different host threads on one device) race on it.
+// calls share it: each call that needs scratch first clears the split-K
+// counters at its start (they must start at zero), and calls whose work
+// overlaps on the GPU (different streams, or different host threads on one
+// device) race on it. A call that the tensor-core or plain kernel takes needs
+// no scratch at all.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -25,6 +27,7 @@ static __device__ __align__(256) unsigned char g_w4_noalloc_scratch[W4_NOALLOC_S
 namespace {
 
 constexpr int kMaxDevNoAlloc = 64;
+constexpr size_t kCounterBytes = 4096;  // the GEMV's split-K counter block at the start of its workspace
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevNoAlloc] = {};
 
@@ -57,7 +60,22 @@ extern "C" w4_status w4_matmul_noalloc(const float* x, int64_t ldx, const uint8_
   const w4host::DeviceInfo* di = nullptr;
   w4_status rc = w4host::current_device(&di);
   if (rc != W4_OK) return rc;
-  const size_t need = w4_matmul_workspace_size(M, K, N);
+  // The split-K scratch is the GEMV's; a call that goes to the tensor-core
+  // kernel (M above 16) or to the plain kernel needs none.
+  w4_desc d = {};
+  d.x = x;
+  d.ldx = ldx;
+  d.qw = qw;
+  d.scales = scales;
+  d.zp = zp;
+  d.y = y;
+  d.ldy = ldy;
+  d.M = M;
+  d.K = K;
+  d.N = N;
+  const char* why = "";
+  const bool gemv = M <= w4host::kTcMinM && w4host::gemv_eligible(d, &why);  // the choice w4_matmul makes
+  const size_t need = gemv ? w4_matmul_workspace_size(M, K, N) : 0;
   if (need > static_cast<size_t>(W4_NOALLOC_SCRATCH_BYTES))
     return w4host::fail(W4_ERR_WORKSPACE,
                         "w4_matmul_noalloc: this shape needs %zu bytes of scratch, more than the %u bytes it holds "
@@ -68,8 +86,11 @@ extern "C" w4_status w4_matmul_noalloc(const float* x, int64_t ldx, const uint8_
   if (rc != W4_OK) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (need > 0) {
-    const cudaError_t e = cudaMemsetAsync(scratch, 0, need, st);
-    if (e != cudaSuccess) return w4host::cuda_fail(e, "clear noalloc scratch");
+    // only the split-K counters must start at zero (the partial sums are
+    // written before they are read); clearing them on every call also resets
+    // a block that a call which timed out left non-zero
+    const cudaError_t e = cudaMemsetAsync(scratch, 0, need < kCounterBytes ? need : kCounterBytes, st);
+    if (e != cudaSuccess) return w4host::cuda_fail(e, "clear noalloc scratch counters");
   }
   return w4_matmul(x, ldx, qw, scales, zp, y, ldy, M, K, N, need > 0 ? scratch : nullptr, need, stream);
 }
