@@ -307,11 +307,12 @@ __global__ void __launch_bounds__(NW * 32, HCfg<MT>::MINB) i8_head_kernel(const 
 
 // A 64-bit key whose unsigned order is the order of (logit, -token): the
 // logit's bits made monotonic (non-negative: sign bit set; negative: all bits
-// flipped) above the complement of the token id, so the maximum key is the
-// largest logit and, among equal logits, the lowest token id. 0 is below
-// every key of a number.
+// flipped; -0 taken as +0) above the complement of the token id, so the
+// maximum key is the largest logit and, among equal logits, the lowest token
+// id. 0 is below every key of a number.
 __device__ __forceinline__ unsigned long long argmax_key(float logit, uint32_t token) {
-  const uint32_t b = __float_as_uint(logit);
+  uint32_t b = __float_as_uint(logit);
+  if (b == 0x80000000u) b = 0u;  // -0 and +0 are the same logit: the lower id must win the tie
   const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
   return (static_cast<unsigned long long>(o) << 32) | static_cast<unsigned long long>(0xFFFFFFFFu - token);
 }

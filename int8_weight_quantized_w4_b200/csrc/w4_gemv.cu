@@ -1083,7 +1083,7 @@ size_t gemv_workspace_bytes(const w4_desc* d, int count, int sms) { return ws_by
 
 // Launch parameters of recent calls, per host thread. A decode loop calls with
 // the same descriptors (weights, inputs and outputs at the same addresses)
-// every step; the parameters are a function of the descriptor bytes, the
+// every step; the parameters are a function of the descriptor fields, the
 // workspace address and the device alone, so an exact match reuses them and
 // skips the tiling, the tensor-map lookups and the role assignment.
 struct PlanEntry {
@@ -1098,6 +1098,20 @@ struct PlanEntry {
   GemvParams prm;
 };
 constexpr int kPlanEntries = 4;
+
+// Field-by-field equality of two descriptor arrays: padding bytes a caller
+// left uninitialised play no part.
+bool same_descs(const w4_desc* a, const w4_desc* b, int count) {
+  for (int i = 0; i < count; ++i) {
+    const w4_desc& p = a[i];
+    const w4_desc& q = b[i];
+    if (p.x != q.x || p.ldx != q.ldx || p.qw != q.qw || p.scales != q.scales || p.zp != q.zp || p.y != q.y ||
+        p.ldy != q.ldy || p.M != q.M || p.K != q.K || p.N != q.N || p.bias != q.bias || p.residual != q.residual ||
+        p.ldr != q.ldr || p.act != q.act || p.reserved != q.reserved)
+      return false;
+  }
+  return true;
+}
 
 w4_status launch_planned(const PlanEntry& e, cudaStream_t st, const DeviceInfo& di) {
   switch (e.mt) {
@@ -1117,7 +1131,7 @@ w4_status launch_gemv(const w4_desc* d, int count, void* ws, size_t ws_size, cud
   ++clock;
   for (int i = 0; i < kPlanEntries; ++i) {
     PlanEntry& e = cache[i];
-    if (e.dev == di.dev && e.count == count && e.ws == ws && std::memcmp(e.descs, d, sizeof(w4_desc) * count) == 0) {
+    if (e.dev == di.dev && e.count == count && e.ws == ws && same_descs(e.descs, d, count)) {
       if (ws_size < e.need) return fail(W4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", e.need, ws_size);
       e.used = clock;
       e.prm.timeout_ns = wait_timeout_ns();

@@ -213,9 +213,11 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
   for (int b = 0; b < m.nb; ++b) {
     const int s = b & 1;
     if (b + 2 < m.nb) load(b + 2, nxt2);
+    // The stage is free once the MMAs that read it two blocks ago are done.
+    // A thread whose bounded wait gives up writes nothing; the barrier below
+    // then takes the whole CTA out of the loop together.
     if (b >= NSTAGE && ok)
       ok = mbar_wait_bounded(&mma_done[s], ((b - NSTAGE) >> 1) & 1, p.timeout_ns, abort_flag, p.err, K_TC, 1);
-    if (!ok) break;
     uint8_t* st = smem + s * STAGE_BYTES;
     uint8_t* a_hi = st;
     uint8_t* a_lo = st + A_PART;
@@ -224,6 +226,7 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
     // x: 128 rows x 32, 16 bytes per thread and pass; the 32 lanes of a warp
     // take 32 consecutive rows, so each store is 4 contiguous core-matrix rows
     // groups (conflict-free)
+    if (ok) {
 #pragma unroll
     for (int i = 0; i < (BM * BK / 4) / NT; ++i) {
       const int r = tid & (BM - 1), q = (tid >> 7) + 2 * i;
@@ -261,10 +264,15 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
         *reinterpret_cast<float4*>(b_lo + off) = make_float4(lv[0], lv[1], lv[2], lv[3]);
       }
     }
+    }  // ok
     fence_async_smem();  // the stores above are read by the tensor core
     tc_fence_before();
-    __syncthreads();
+    const bool any_failed = __syncthreads_or(!ok) != 0;  // one decision for the whole CTA
     tc_fence_after();
+    if (any_failed) {
+      ok = false;
+      break;
+    }
     if (tid == 0) {
       const uint32_t ah = smem_u32(a_hi), al = smem_u32(a_lo), bh = smem_u32(b_hi), bl = smem_u32(b_lo);
 #pragma unroll
@@ -288,6 +296,9 @@ __global__ void __launch_bounds__(NT, 1) w4_tc_kernel(const __grid_constant__ Tc
     const bool done = mbar_wait_bounded(&mma_done[b & 1], (b >> 1) & 1, p.timeout_ns, abort_flag, p.err, K_TC, 2);
     ok = ok && done;
   }
+  // the epilogue's tensor-memory loads are warp-collective: every thread
+  // takes the same decision
+  ok = __syncthreads_and(ok) != 0;
   tc_fence_after();
   if (ok && issued == m.nb) {
     const int quad = warp & 3;  // TMEM lanes 32 quad .. 32 quad + 31 = rows of the tile

@@ -64,6 +64,23 @@ def test_argmax_ties_go_to_the_lowest_token():
     assert int(tok.item()) == 123 and float(best.item()) == 0.5 * 100 * K
 
 
+def test_argmax_signed_zero_tie_goes_to_the_lowest_token():
+    """-0 and +0 are equal logits: the lower token id wins even when its
+    logit is the negative zero (a zero column under a negative scale)."""
+    K, V = 32, 1000
+    table = np.full((K, V), -20, np.int8)
+    table[:, 123] = 0
+    table[:, 700] = 0
+    s = np.full(V, 0.5, np.float32)
+    s[123] = -0.5  # 0 * -0.5 = -0
+    h = np.ones((1, K), np.float32)
+    for M in (1, 3):  # the fused rows kernel and the workspace path
+        hm = np.repeat(h, M, axis=0)
+        tok, best = w4().i8_head_argmax(dev(hm), dev(table), dev(s), K, V)
+        torch().cuda.synchronize()
+        assert list(tok.cpu().numpy()) == [123] * M and np.all(best.cpu().numpy() == 0.0)
+
+
 def test_argmax_leaves_the_counter_block_zero():
     """Calls share one workspace; its first 4 KB (the split-K counters of
     every kernel) must be zero after each of them."""
