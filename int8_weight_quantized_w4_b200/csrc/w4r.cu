@@ -30,17 +30,24 @@
 //   multiple of 8 gs) are zero in the repacked buffer and never written.
 //
 // GEMV design (sm_100a, M = 1):
-//  * A CTA is 4 warps; each warp owns one group (8 gs columns, all of K), so
-//    every output column is summed by one warp with no partial sums in
-//    memory. For the GPT-2 and 3.8B shapes every group is 96 atoms (15.7 KB)
-//    or, for K = 8192, 256 atoms.
-//  * Each warp streams its group through a ring of 3 stages of one round,
-//    with one bulk copy per round issued by its lane 0 (no multicast); for
-//    A <= 3 the whole group is requested at the CTA's first instruction.
-//  * The CTA stages x in shared memory as [row quad c][block b][4 floats] so
-//    that lanes reading different blocks hit different banks.
+//  * One persistent CTA per SM takes an equal share of the launch's groups
+//    (all matrices' groups in one flat list; CTA c takes [c T / G, (c+1) T / G)).
+//    Each of its 16 warps is an independent stream: warp w owns the groups
+//    lo + w, lo + w + 16, ... of that share, so every output column is summed
+//    inside one warp, with no partial sums in memory and no workspace. For
+//    the GPT-2 shapes a group is 96 atoms (15.7 KB) and a CTA about 24 groups.
+//  * A warp streams its rounds, group after group, through a ring of 2
+//    stages; its lane 0 issues one bulk copy per round (no multicast) as soon
+//    as the stage it refills has been read, so the SM keeps up to 32 rounds
+//    (168 KB) of its stream in flight. Four warps per scheduler (measured
+//    against 3 warps x 3 stages and 2 x 4: 15.7 vs 16.2 and 18.8 us for the
+//    GPT-2 body) hide more of the decode's dependency stalls.
+//  * The CTA stages the x of every matrix its share touches in shared memory
+//    as [row quad c][block b][4 floats], so lanes reading different blocks hit
+//    different banks (the host splits a launch whose shares would need more
+//    than 8192 floats).
 //  * The launch lets the next launch in the stream start early (programmatic
-//    dependent launch): a CTA requests its weight bytes before it waits for
+//    dependent launch): a CTA requests its first rounds before it waits for
 //    the previous launch to finish, and reads x / writes y only after that
 //    wait. The weights are constants of the model; x and y may belong to the
 //    previous launch.
@@ -69,10 +76,12 @@ constexpr int ROUND_BYTES = 5248;
 constexpr int NIB_BYTES = 4096;
 constexpr int SC_BYTES = 1024;
 constexpr int ROUND_WORDS = ROUND_BYTES / 4;  // 1312
-constexpr int RW = 4;                         // warps per CTA
-constexpr int NST = 3;                        // stages per warp
+constexpr int PW = 16;                        // warps per CTA, each its own stream
+constexpr int PST = 2;                        // stages per warp
 constexpr int RCAP = 64;                      // matrices per launch
-constexpr int STAGE_SMEM = RW * NST * ROUND_BYTES;
+constexpr int XCAP = 8192;                    // floats of x a CTA can hold
+constexpr int STAGE_SMEM = PW * PST * ROUND_BYTES;
+constexpr int SMEM_BYTES = STAGE_SMEM + XCAP * 4 + PW * PST * 8 + PW * 4;
 
 struct RMat {
   const uint8_t* wr;
@@ -83,7 +92,7 @@ struct RMat {
   int64_t ldr;
   int32_t K;
   int32_t N;
-  int32_t cta0;     // first CTA of this matrix in the launch
+  int32_t g0;       // first group of this matrix in the launch's flat list
   int32_t ngroups;  // groups of 8 gs columns
   int32_t act;
   int32_t gsl;      // log2(gs)
@@ -92,7 +101,7 @@ struct RMat {
 struct RParams {
   RMat m[RCAP];
   int32_t count;
-  int32_t x_floats;  // shared-memory floats reserved for x
+  int32_t T;  // groups of the launch
   ErrorWord* err;
   uint64_t timeout_ns;
 };
@@ -105,6 +114,20 @@ __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepc
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Range of groups [lo, hi) of CTA c out of G (T * G < 2^31 by the host).
+__device__ __forceinline__ int range_lo(int c, int T, int G) { return (c * T) / G; }
+
+// Matrix holding flat group gg: the last one whose first group is <= gg.
+__device__ __forceinline__ int mat_of(const RParams& p, int gg) {
+  int lo = 0, hi = p.count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.m[mid].g0 <= gg) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 // One atom: 8 columns x 32 rows for this lane, accumulated into acc[0..7].
 // st: the stage; xb: x of the atom's block in the [c][b][4] layout, c-th
 // quad at xb + c * xq floats.
@@ -114,13 +137,14 @@ __device__ __forceinline__ void atom_m1(const uint8_t* st, int lane, const float
   float2 nz[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float z = -magic_nib(i < 4 ? zw : (zw >> 16), i & 3);
+    // -(2^23 + zp 16^j): the nibble in the mantissa of -2^23
+    const float z = __uint_as_float(0xCB000000u | ((i < 4 ? zw : (zw >> 16)) & (0xFu << (4 * (i & 3)))));
     nz[i] = make_float2(z, z);
   }
   float2 P[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) P[i] = make_float2(0.f, 0.f);
-#pragma unroll 2
+#pragma unroll
   for (int c = 0; c < 8; ++c) {
     const uint4 wv = *reinterpret_cast<const uint4*>(st + c * 512 + lane * 16);
     const float4 x4 = *reinterpret_cast<const float4*>(xb + c * xq);
@@ -148,133 +172,192 @@ __device__ __forceinline__ void atom_m1(const uint8_t* st, int lane, const float
   for (int i = 0; i < 8; ++i) acc[i] = fmaf(P[i].x + P[i].y, sv[i] * inv_slot_scale(i & 3), acc[i]);
 }
 
-__global__ void __launch_bounds__(RW * 32, 3) w4r_gemv_m1_kernel(const __grid_constant__ RParams p) {
+// The rounds one warp streams, in order: its groups lo + warp + PW t, each
+// of A rounds. Producer (lane 0) and consumers walk the same sequence.
+struct RoundWalk {
+  int t, r, ngw;  // group ordinal of this warp, round in it, groups of this warp
+  int g, A;       // matrix of the current group, its rounds per group
+  const uint8_t* base;
+};
+
+__device__ __forceinline__ void walk_group(RoundWalk& w, const RParams& p, int lo, int warp) {
+  const int gg = lo + warp + PW * w.t;
+  while (w.g + 1 < p.count && p.m[w.g + 1].g0 <= gg) ++w.g;
+  const RMat& m = p.m[w.g];
+  w.A = ((m.K >> 5) << m.gsl) >> 5;
+  w.base = m.wr + static_cast<int64_t>(gg - m.g0) * w.A * ROUND_BYTES;
+}
+
+__global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_constant__ RParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const int lo = range_lo(blockIdx.x, p.T, G);
+  const int hi = range_lo(blockIdx.x + 1, p.T, G);
+  const int ngw = hi - lo > warp ? (hi - lo - warp + PW - 1) / PW : 0;  // groups of this warp
 
-  // matrix of this CTA: the last one whose first CTA is at or before it
-  int g = 0;
-  {
-    int lo = 0, hi = p.count - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (p.m[mid].cta0 <= static_cast<int>(blockIdx.x)) lo = mid;
-      else hi = mid - 1;
-    }
-    g = lo;
-  }
-  const RMat& m = p.m[g];
-  const int K = m.K;
-  const int nb = K >> 5;
-  const int gsl = m.gsl;
-  const int A = (nb << gsl) >> 5;  // rounds of a group
-  const int group = (static_cast<int>(blockIdx.x) - m.cta0) * RW + warp;
-  const bool active = group < m.ngroups;
-
-  uint8_t* stg = smem + warp * (NST * ROUND_BYTES);
+  uint8_t* stg = smem + warp * (PST * ROUND_BYTES);
   float* xs = reinterpret_cast<float*>(smem + STAGE_SMEM);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + STAGE_SMEM + p.x_floats * 4) + warp * NST;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + STAGE_SMEM + p.x_floats * 4 + RW * NST * 8) + warp;
-  const uint8_t* src = m.wr + static_cast<int64_t>(group) * A * ROUND_BYTES;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + STAGE_SMEM + XCAP * 4) + warp * PST;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + STAGE_SMEM + XCAP * 4 + PW * PST * 8) + warp;
 
-  // ---- weights first: they do not depend on the previous launch
-  int issued = 0;  // rounds requested (lane 0)
-  if (active && lane == 0) {
-    for (int s = 0; s < NST; ++s) mbar_init(&bar[s], 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-    const int n0 = min(A, NST);
-    for (int r = 0; r < n0; ++r) {
-      mbar_arrive_expect_tx(&bar[r], ROUND_BYTES);
-      bulk_g2s(stg + r * ROUND_BYTES, src + static_cast<int64_t>(r) * ROUND_BYTES, ROUND_BYTES, &bar[r]);
+  // ---- x into L2 now: a cache hint only (the values are read after the
+  // wait), so that the staging below does not queue behind weight bytes
+  if (threadIdx.x == 0) {
+    const int g1 = hi > lo ? mat_of(p, hi - 1) : mat_of(p, lo);
+    for (int g = mat_of(p, lo); g <= g1; ++g)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.m[g].x), "r"(p.m[g].K * 4) : "memory");
+  }
+  // ---- the first round of every warp before the wait: the weights do not
+  // depend on the previous launch, so they stream while it finishes
+  const int gfirst = mat_of(p, lo);
+  RoundWalk iw{0, 0, ngw, gfirst, 0, nullptr};  // issue cursor, kept in step by every lane
+  int issued = 0;
+  if (ngw > 0) {
+    walk_group(iw, p, lo, warp);
+    if (lane == 0) {
+      for (int s = 0; s < PST; ++s) mbar_init(&bar[s], 1);
+      *abort_flag = 0;
+      fence_mbar_init();
+      mbar_arrive_expect_tx(&bar[0], ROUND_BYTES);
+      bulk_g2s(stg, iw.base + static_cast<int64_t>(iw.r) * ROUND_BYTES, ROUND_BYTES, &bar[0]);
     }
-    issued = n0;
+    issued = 1;
+    if (++iw.r == iw.A) {
+      iw.r = 0;
+      if (++iw.t < ngw) walk_group(iw, p, lo, warp);
+    }
   }
   __syncwarp();
   pdl_launch_dependents();
   pdl_wait();  // x and y may be the previous launch's
 
-  // ---- x of this CTA's matrix into shared memory, [quad c][block b][4]
-  for (int i = threadIdx.x; i < (K >> 2); i += RW * 32) {
-    const int b = i >> 3, c = i & 7;
-    cp_async_16(xs + (c * nb + b) * 4, m.x + 4 * i, 16);
+  // ---- x of every matrix this CTA's range touches, [quad c][block b][4]
+  // each: requested before the rest of the weights, which would otherwise
+  // queue ahead of it
+  const int glast = hi > lo ? mat_of(p, hi - 1) : gfirst;
+  {
+    int xo = 0;
+    for (int g = gfirst; g <= glast; ++g) {
+      const int K = p.m[g].K;
+      const int nb = K >> 5;
+      const float* xg = p.m[g].x;
+      for (int i = threadIdx.x; i < (K >> 2); i += PW * 32) {
+        const int b = i >> 3, c = i & 7;
+        cp_async_16(xs + xo + (c * nb + b) * 4, xg + 4 * i, 16);
+      }
+      xo += K;
+    }
   }
   cp_async_commit();
   cp_async_wait_group<0>();
   __syncthreads();
-  if (!active) return;
+  // ---- the warp's other stages, once x is in: the first round is already
+  // here or in flight, so the stream does not stall meanwhile
+  for (int s = 1; s < PST && iw.t < ngw; ++s) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar[s], ROUND_BYTES);
+      bulk_g2s(stg + s * ROUND_BYTES, iw.base + static_cast<int64_t>(iw.r) * ROUND_BYTES, ROUND_BYTES, &bar[s]);
+    }
+    ++issued;
+    if (++iw.r == iw.A) {
+      iw.r = 0;
+      if (++iw.t < ngw) walk_group(iw, p, lo, warp);
+    }
+  }
+  if (ngw == 0) return;
 
   uint32_t kMagic;  // 0x4B000000 (the bits of 2^23) held in a register
   asm("mov.b32 %0, 0x4B000000;" : "=r"(kMagic));
-  const int gs = 1 << gsl;
-  const int strip = lane & (gs - 1);
-  const int phase = lane >> gsl;
-  const int pstride = 32 >> gsl;
-  const int xq = nb * 4;  // floats between row quads of x
-  float acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 
   bool ok = true;
   int s = 0;
   uint32_t par = 0;
+  int g = gfirst;
+  int xo = 0;  // x offset of matrix g in shared memory
 #pragma unroll 1
-  for (int r = 0; r < A; ++r) {
-    ok = mbar_wait_bounded(&bar[s], par, p.timeout_ns, abort_flag, p.err, K_GEMVR, 1);
-    if (__any_sync(0xffffffffu, !ok)) {
-      ok = false;
-      break;
+  for (int t = 0; t < ngw && ok; ++t) {
+    const int gg = lo + warp + PW * t;
+    while (g < glast && p.m[g + 1].g0 <= gg) {
+      xo += p.m[g].K;
+      ++g;
     }
-    const int b = phase + r * pstride;
-    atom_m1(stg + s * ROUND_BYTES, lane, xs + b * 4, xq, kMagic, acc);
-    __syncwarp();
-    if (lane == 0 && issued < A) {  // refill this stage with the round NST ahead
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&bar[s], ROUND_BYTES);
-      bulk_g2s(stg + s * ROUND_BYTES, src + static_cast<int64_t>(issued) * ROUND_BYTES, ROUND_BYTES, &bar[s]);
-      ++issued;
+    const RMat& m = p.m[g];
+    const int nb = m.K >> 5;
+    const int gsl = m.gsl;
+    const int A = (nb << gsl) >> 5;
+    const int gs = 1 << gsl;
+    const int phase = lane >> gsl;
+    const int pstride = 32 >> gsl;
+    const float* xw = xs + xo + phase * 4;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 1
+    for (int r = 0; r < A; ++r) {
+      ok = mbar_wait_bounded(&bar[s], par, p.timeout_ns, abort_flag, p.err, K_GEMVR, 1);
+      if (__any_sync(0xffffffffu, !ok)) {
+        ok = false;
+        break;
+      }
+      atom_m1(stg + s * ROUND_BYTES, lane, xw + r * pstride * 4, nb * 4, kMagic, acc);
+      __syncwarp();
+      if (iw.t < ngw) {  // refill this stage with the round PST ahead (the walk is warp-uniform)
+        if (lane == 0) {
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&bar[s], ROUND_BYTES);
+          bulk_g2s(stg + s * ROUND_BYTES, iw.base + static_cast<int64_t>(iw.r) * ROUND_BYTES, ROUND_BYTES, &bar[s]);
+        }
+        ++issued;
+        if (++iw.r == iw.A) {
+          iw.r = 0;
+          if (++iw.t < ngw) walk_group(iw, p, lo, warp);
+        }
+      }
+      if (++s == PST) {
+        s = 0;
+        par ^= 1u;
+      }
     }
-    if (++s == NST) {
-      s = 0;
-      par ^= 1u;
+    if (!ok) break;
+
+    // ---- the lanes of a strip: butterfly over the phase bits
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1)
+      if (off >= gs) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+      }
+    const int col = (((gg - m.g0) << gsl) + (lane & (gs - 1))) * 8;
+    if (phase == 0 && col < m.N) {
+      float* yp = m.y + col;
+      const Epi epi{m.bias, m.res, m.ldr, m.act, 0};
+      float v[8];
+      if (epi_active(epi)) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = epi_apply(acc[i], epi, 0, col + i);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = acc[i];
+      }
+      if ((reinterpret_cast<uintptr_t>(yp) & 15) == 0) {
+        reinterpret_cast<float4*>(yp)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4*>(yp)[1] = make_float4(v[4], v[5], v[6], v[7]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) yp[i] = v[i];
+      }
     }
   }
 
-  if (!ok) {
+  if (!ok && lane == 0) {
     // copies still in flight must land before the CTA exits: wait (bounded)
     // for the last fill of every stage
-    if (lane == 0)
-      for (int st = 0; st < NST; ++st) {
-        const int fills = issued > st ? (issued - st + NST - 1) / NST : 0;
-        if (fills > 0) mbar_wait_bounded(&bar[st], (fills - 1) & 1, p.timeout_ns, nullptr, p.err, K_GEMVR, 2);
-      }
-    return;
-  }
-
-  // ---- the lanes of a strip: butterfly over the phase bits
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    for (int off = gs; off < 32; off <<= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
-  if (phase != 0) return;
-  const int col = ((group << gsl) + strip) * 8;
-  if (col >= m.N) return;
-  float* yp = m.y + col;
-  const Epi epi{m.bias, m.res, m.ldr, m.act, 0};
-  float v[8];
-  if (epi_active(epi)) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = epi_apply(acc[i], epi, 0, col + i);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = acc[i];
-  }
-  if ((reinterpret_cast<uintptr_t>(yp) & 15) == 0) {
-    reinterpret_cast<float4*>(yp)[0] = make_float4(v[0], v[1], v[2], v[3]);
-    reinterpret_cast<float4*>(yp)[1] = make_float4(v[4], v[5], v[6], v[7]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) yp[i] = v[i];
+    for (int st = 0; st < PST; ++st) {
+      const int fills = issued > st ? (issued - st + PST - 1) / PST : 0;
+      if (fills > 0) mbar_wait_bounded(&bar[st], (fills - 1) & 1, p.timeout_ns, nullptr, p.err, K_GEMVR, 2);
+    }
   }
 }
 
@@ -414,23 +497,48 @@ w4_status check_rdesc(const w4r_desc& d, RepackGeom* g) {
   if (d.x == nullptr || d.wr == nullptr) return fail(W4_ERR_NULL, "x and wr must not be NULL");
   if (!aligned_to(d.x, 16)) return fail(W4_ERR_ALIGN, "the streaming-layout GEMV needs x 16-byte aligned");
   if (!aligned_to(d.wr, 16)) return fail(W4_ERR_ALIGN, "the repacked weight must be 16-byte aligned");
-  if (d.K > 32768) return fail(W4_ERR_SHAPE, "the streaming-layout GEMV takes K <= 32768 (K=%lld)", (long long)d.K);
+  if (d.K > XCAP) return fail(W4_ERR_SHAPE, "the streaming-layout GEMV takes K <= %d (K=%lld)", XCAP, (long long)d.K);
   geom_of(d.K, d.N, g);
   return W4_OK;
 }
 
-int rsmem_bytes(int x_floats) { return STAGE_SMEM + x_floats * 4 + RW * NST * 8 + RW * 4; }
+// x floats that CTA c of G must hold: the sum of K over the matrices its
+// range of groups touches.
+int64_t max_x_need(const w4r_desc* d, const RepackGeom* geo, int count, int64_t T, int G) {
+  int64_t worst = 0;
+  int64_t g0 = 0;
+  int gi = 0;
+  for (int c = 0; c < G; ++c) {
+    const int64_t lo = c * T / G, hi = (c + 1) * T / G;
+    if (hi <= lo) continue;
+    while (gi + 1 < count && g0 + geo[gi].ngroups <= lo) g0 += geo[gi++].ngroups;
+    int64_t need = 0, gg0 = g0;
+    for (int gj = gi; gj < count && gg0 < hi; gg0 += geo[gj++].ngroups) need += d[gj].K;
+    worst = std::max(worst, need);
+  }
+  return worst;
+}
 
 w4_status launch_rgroup(const w4r_desc* d, const RepackGeom* geo, int count, cudaStream_t st,
                         const w4host::DeviceInfo& di) {
   using namespace w4host;
+  int64_t T = 0;
+  for (int i = 0; i < count; ++i) T += geo[i].ngroups;
+  const int G = static_cast<int>(std::min<int64_t>(di.sms, T));
+  // every CTA stages the x of each matrix its range touches: split the
+  // launch until that fits its shared memory
+  if (count > 1 && max_x_need(d, geo, count, T, G) > XCAP) {
+    const int h = count / 2;
+    const w4_status rc = launch_rgroup(d, geo, h, st, di);
+    if (rc != W4_OK) return rc;
+    return launch_rgroup(d + h, geo + h, count - h, st, di);
+  }
+  if (T * G >= (int64_t(1) << 31)) return fail(W4_ERR_SHAPE, "too many groups for one launch (%lld)", (long long)T);
   RParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  int cta = 0;
-  int xf = 0;
+  int g0 = 0;
   for (int i = 0; i < count; ++i) {
     RMat& m = prm.m[i];
-    const RepackGeom& g = geo[i];
     m.wr = static_cast<const uint8_t*>(d[i].wr);
     m.x = d[i].x;
     m.y = d[i].y;
@@ -439,29 +547,27 @@ w4_status launch_rgroup(const w4r_desc* d, const RepackGeom* geo, int count, cud
     m.ldr = d[i].ldr;
     m.K = static_cast<int32_t>(d[i].K);
     m.N = static_cast<int32_t>(d[i].N);
-    m.cta0 = cta;
-    m.ngroups = g.ngroups;
+    m.g0 = g0;
+    m.ngroups = geo[i].ngroups;
     m.act = d[i].act;
-    m.gsl = g.gsl;
-    cta += (g.ngroups + RW - 1) / RW;
-    xf = std::max(xf, m.K);
+    m.gsl = geo[i].gsl;
+    g0 += geo[i].ngroups;
   }
   prm.count = count;
-  prm.x_floats = xf;
+  prm.T = static_cast<int32_t>(T);
   prm.err = di.err;
   prm.timeout_ns = wait_timeout_ns();
-  const int smem = rsmem_bytes(xf);
   static int configured[64] = {};
-  if (di.dev < 64 && configured[di.dev] < smem) {
-    const cudaError_t e = cudaFuncSetAttribute(w4r_gemv_m1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               rsmem_bytes(32768));
+  if (di.dev < 64 && !configured[di.dev]) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(w4r_gemv_m1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(w4r_gemv)");
-    configured[di.dev] = rsmem_bytes(32768);
+    configured[di.dev] = 1;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(cta));
-  cfg.blockDim = dim3(RW * 32);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.gridDim = dim3(static_cast<unsigned>(G));
+  cfg.blockDim = dim3(PW * 32);
+  cfg.dynamicSmemBytes = static_cast<size_t>(SMEM_BYTES);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
