@@ -171,15 +171,18 @@ W4_API w4_status w4_matmul_path(const float* x, int64_t ldx, const uint8_t* qw, 
  * and outputs are the caller's, exactly as for w4_matmul; the split-K scratch
  * comes from one array of W4_NOALLOC_SCRATCH_BYTES inside this library,
  * which every GPU that loads the library keeps until the process exits.
- * - Shapes whose scratch need (w4_matmul_workspace_size) exceeds that size
+ * - The scratch is the split-K GEMV's (M <= 16); a call that w4_matmul sends
+ *   to the tensor-core kernel (M > 16) or to the plain kernel needs none.
+ *   Shapes whose scratch need (w4_matmul_workspace_size) exceeds the array
  *   are refused with W4_ERR_WORKSPACE. The need grows with M and with the
- *   number of SMs the call keeps busy (4 KB + SMs x M' x 4 KB, M' = M
- *   rounded up to 1, 2, 4 or 8): on a 148-SM B200 every M <= 2 fits (at
- *   most 1.2 MB), while M from 3 to 16 fits only for weights too small to
- *   fill the GPU.
- * - Each call clears the part of the array it uses, then runs as w4_matmul.
- *   Calls share the array, so calls that overlap on the GPU (other streams,
- *   other host threads on the same device) race: serialise them.
+ *   number of SMs the call keeps busy (4 KB + SMs x M' x 4 KB, M' = M rounded
+ *   up to 1, 2, 4 or 8): on a 148-SM B200 every M <= 2 fits (at most
+ *   1.2 MB), while M from 3 to 16 fits only for weights too small to fill
+ *   the GPU.
+ * - Each call that needs scratch first clears the split-K counters at its
+ *   start, then runs as w4_matmul. Calls share the array, so calls that
+ *   overlap on the GPU (other streams, other host threads on the same
+ *   device) race: serialise them.
  * - The first call on a device looks up the array's device address; make
  *   that first call before any stream capture.
  * Calls no allocating routine. */
@@ -238,7 +241,7 @@ W4_API w4_status w4_repack_restore(const void* wr, int64_t K, int64_t N, uint8_t
 /* One decode matmul on a repacked weight: y[1, N] = act(x[1, K] . W + bias)
  * + residual, the fields and the epilogue as in w4_desc (ldx / ldy / ldr are
  * not used: one row). Requires M == 1 (W4_ERR_SHAPE otherwise), K % 32 == 0,
- * K <= 32768, N % 8 == 0, x and wr 16-byte aligned, y / bias / residual
+ * K <= 8192, N % 8 == 0, x and wr 16-byte aligned, y / bias / residual
  * 4-byte aligned. No workspace: every output column is summed inside one
  * warp. reserved must be 0. */
 typedef struct w4r_desc {
@@ -291,6 +294,50 @@ W4_API w4_status i8_head_logits_path(const float* h, int64_t ldh, const int8_t* 
                                      const float* scales, float* logits, int64_t ldl, int64_t M,
                                      int64_t K, int64_t V, void* workspace, size_t workspace_bytes,
                                      w4_path path, void* stream);
+
+/* The streaming layout of the int8 head: the page's table bytes and scales
+ * ("ONNX export, quantization and the browser runtime", section
+ * "Quantization (train/quantize.py)", step 3) reordered once at load time
+ * into the order in which the M = 1 head GEMV streams them, one contiguous
+ * run of bytes per warp, and biased to unsigned (code XOR 0x80). Nothing is
+ * rounded: i8_head_repack_restore gives back the page's table and scales
+ * exactly.
+ *
+ * Layout, K % 16 == 0, nb = K / 16, gs = 32 / gcd(nb, 32), A = gs * nb / 32:
+ * groups of 8 gs token columns (all K rows) in column order; a group is A
+ * rounds of 4096 bytes followed by its 8 gs scales (fp32). In round r of
+ * group G, lane l owns strip s = l % gs (columns c0 = 8 (G gs + s) ..
+ * c0 + 7) and block b = l / gs + r * (32 / gs) (rows 16 b .. 16 b + 15);
+ * the byte of row 16 b + 2 c + e, column c0 + 4 h + i sits at
+ * c * 512 + l * 16 + (2 e + h) * 4 + i. Columns at or past V hold code 0 and
+ * scale 0. i8_head_repacked_bytes() is the size (0 for a shape the layout
+ * does not take: K % 16 != 0, K > 8192, V < 1). */
+W4_API size_t i8_head_repacked_bytes(int64_t K, int64_t V);
+
+/* Page format (table [K, V] with row stride ldt >= V, any alignment;
+ * scales [V] fp32, 4-byte aligned) -> streaming layout tr
+ * (i8_head_repacked_bytes(K, V) bytes, 16-byte aligned), on the GPU. */
+W4_API w4_status i8_head_repack(const int8_t* table, int64_t ldt, const float* scales, int64_t K, int64_t V,
+                                void* tr, void* stream);
+
+/* Streaming layout -> page format (the exact inverse of i8_head_repack). */
+W4_API w4_status i8_head_repack_restore(const void* tr, int64_t K, int64_t V, int8_t* table, int64_t ldt,
+                                        float* scales, void* stream);
+
+/* logits[v] = s_v * sum_k h[k] T[k, v] for ONE last-position row h (K fp32,
+ * 16-byte aligned) on a repacked head; logits: V fp32, 4-byte aligned, fully
+ * overwritten. No workspace. Like w4r_matmul_grouped, the launch may start
+ * streaming the table before the previous work on the stream has finished;
+ * h is read and the logits written only after it has. */
+W4_API w4_status i8r_head_logits(const float* h, const void* tr, int64_t K, int64_t V, float* logits,
+                                 void* stream);
+
+/* Greedy decoding on a repacked head: *token = argmax_v of exactly the
+ * logits i8r_head_logits computes (ties to the lowest id; -0 equals +0),
+ * *best_logit (may be NULL) = that logit; the logits are not written. keys:
+ * 8 bytes of device memory (8-byte aligned) that the call clears and uses. */
+W4_API w4_status i8r_head_argmax(const float* h, const void* tr, int64_t K, int64_t V, int32_t* token,
+                                 float* best_logit, void* keys, void* stream);
 
 /* Greedy decoding on the head: tokens[m] = argmax_v logits[m, v] (ties to
  * the lowest token id), best_logits[m] = that logit when best_logits is not

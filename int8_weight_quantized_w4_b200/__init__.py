@@ -12,6 +12,8 @@ Operations (see include/w4.h for layouts and error behaviour):
   w4_repack(qw, scales, zp, K, N)           the weight in the streaming layout (once, at load)
   w4r_matmul(x, wr, K, N) / _grouped        decode (M = 1) on repacked weights
   i8_head_logits(h, table, scales, K, V)    last-position logits, int8 head
+  i8_head_repack(table, scales, K, V)       the head in the streaming layout (once, at load)
+  i8r_head_logits(h, tr, K, V) / _argmax    M = 1 head on the repacked table
   w4_quantize(w, block, scale_type)         the dq4 quantiser (GPU)
   i8_quantize_head(w)                       the embedding_int8 quantiser (GPU)
   pack_nibbles / unpack_nibbles             host-side UINT4 packing
@@ -277,6 +279,54 @@ def i8_head_argmax(h, table, scales, K: int, V: int, ldt: int | None = None, str
                               _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream_handle(stream))
     _check(st, "i8_head_argmax")
     return tokens, best
+
+
+def i8_head_repacked_bytes(K: int, V: int) -> int:
+    return int(lib().i8_head_repacked_bytes(K, V))
+
+
+def i8_head_repack(table, scales, K: int, V: int, ldt: int | None = None, stream=None):
+    """The int8 head (page format) in the streaming layout the M = 1 head
+    GEMV reads: a uint8 device tensor of i8_head_repacked_bytes(K, V) bytes."""
+    torch = _torch()
+    ldt = V if ldt is None else ldt
+    n = i8_head_repacked_bytes(K, V)
+    if n == 0:
+        raise ValueError(f"the streaming head does not take K={K}, V={V}")
+    out = torch.empty(n, dtype=torch.uint8, device=table.device)
+    _check(lib().i8_head_repack(_ptr(table), ldt, _ptr(scales), K, V, _ptr(out), _stream_handle(stream)),
+           "i8_head_repack")
+    return out
+
+
+def i8_head_repack_restore(tr, K: int, V: int, stream=None):
+    """(table [K, V] int8, scales [V] fp32) of a repacked head."""
+    torch = _torch()
+    table = torch.empty((K, V), dtype=torch.int8, device=tr.device)
+    sc = torch.empty(V, dtype=torch.float32, device=tr.device)
+    _check(lib().i8_head_repack_restore(_ptr(tr), K, V, _ptr(table), V, _ptr(sc), _stream_handle(stream)),
+           "i8_head_repack_restore")
+    return table, sc
+
+
+def i8r_head_logits(h, tr, K: int, V: int, logits=None, stream=None):
+    """logits [1, V] of one last-position row h on a repacked head."""
+    torch = _torch()
+    if logits is None:
+        logits = torch.empty((1, V), dtype=torch.float32, device=h.device)
+    _check(lib().i8r_head_logits(_ptr(h), _ptr(tr), K, V, _ptr(logits), _stream_handle(stream)), "i8r_head_logits")
+    return logits
+
+
+def i8r_head_argmax(h, tr, K: int, V: int, stream=None):
+    """(token int32 [1], best logit fp32 [1]) of one row h on a repacked head."""
+    torch = _torch()
+    tok = torch.empty(1, dtype=torch.int32, device=h.device)
+    best = torch.empty(1, dtype=torch.float32, device=h.device)
+    keys = torch.empty(1, dtype=torch.int64, device=h.device)
+    _check(lib().i8r_head_argmax(_ptr(h), _ptr(tr), K, V, _ptr(tok), _ptr(best), _ptr(keys), _stream_handle(stream)),
+           "i8r_head_argmax")
+    return tok, best
 
 
 def i8_embed_lookup(table, scales, tokens, K: int, V: int, ldt: int | None = None, out=None, stream=None):

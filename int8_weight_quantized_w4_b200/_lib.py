@@ -88,6 +88,13 @@ SIGNATURES = {
                                     C.c_void_p]),
     "w4r_matmul": (C.c_int, [C.POINTER(W4RDesc), C.c_void_p]),
     "w4r_matmul_grouped": (C.c_int, [C.POINTER(W4RDesc), C.c_int32, C.c_void_p]),
+    "i8_head_repacked_bytes": (C.c_size_t, [C.c_int64, C.c_int64]),
+    "i8_head_repack": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),
+    "i8_head_repack_restore": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p,
+                                         C.c_void_p]),
+    "i8r_head_logits": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),
+    "i8r_head_argmax": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p,
+                                  C.c_void_p, C.c_void_p]),
     "i8_head_workspace_size": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int64]),
     "i8_head_argmax_workspace_size": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int64]),
     "i8_head_argmax": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_int64,
