@@ -233,8 +233,9 @@ class Workload:
                                      for i, (_, K, N) in enumerate(self.shapes)])
             t = table if r == 0 else table.clone()
             s = hsc if r == 0 else hsc.clone()
+            tr = w4.i8_head_repack(t, s, HEAD_K, HEAD_V)  # the head in its streaming layout (once, at load)
             # the descriptors hold raw pointers: keep every tensor they name alive
-            self.copies.append((descs, t, s, ws, rdescs, wrs))
+            self.copies.append((descs, t, s, ws, rdescs, wrs, tr))
         need = max(w4.w4_matmul_grouped_workspace_size(self.copies[0][0]),
                    w4.i8_head_workspace_size(1, HEAD_K, HEAD_V))
         self.ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
@@ -257,6 +258,14 @@ class Workload:
             raise RuntimeError(f"w4_matmul_grouped failed: {st} {self.lib.w4_last_error()}")
 
     def head(self, r: int, stream_handle: int):
+        """The int8 head on the last position, repacked (the product path)."""
+        tr = self.copies[r][6]
+        st = self.lib.i8r_head_logits(self.h.data_ptr(), tr.data_ptr(), HEAD_K, HEAD_V, self.logits.data_ptr(),
+                                      stream_handle)
+        if st != 0:
+            raise RuntimeError(f"i8r_head_logits failed: {st} {self.lib.w4_last_error()}")
+
+    def head_page_format(self, r: int, stream_handle: int):
         _, t, s = self.copies[r][:3]
         st = self.lib.i8_head_logits(self.h.data_ptr(), HEAD_K, t.data_ptr(), HEAD_V, s.data_ptr(),
                                      self.logits.data_ptr(), HEAD_V, 1, HEAD_K, HEAD_V, self.ws.data_ptr(),
@@ -332,10 +341,12 @@ def run_ours(args, world, rank, local):
     g_body = capture([wl.body])
     g_head = capture([wl.head])
     g_page = capture([wl.body_page_format])
+    g_hpage = capture([wl.head_page_format])
     n_step = reps_for(g_step, args.seconds)
     n_body = reps_for(g_body, args.seconds / 2)
     n_head = reps_for(g_head, args.seconds / 2)
     n_page = reps_for(g_page, args.seconds / 4)
+    n_hpage = reps_for(g_hpage, args.seconds / 4)
     sampler = ClockSampler(gpu_id(local if world > 1 else 0))
     sampler.start()
     time.sleep(0.2)
@@ -343,10 +354,11 @@ def run_ours(args, world, rank, local):
     body_avg = timed(g_body, n_body) / (K * n_body)
     head_avg = timed(g_head, n_head) / (K * n_head)
     page_avg = timed(g_page, n_page) / (K * n_page)
+    hpage_avg = timed(g_hpage, n_hpage) / (K * n_hpage)
     clocks = sampler.stop()
     steps_timed = K * n_step
     ms_step = total_ms / steps_timed
-    del g_step, g_body, g_head, g_page
+    del g_step, g_body, g_head, g_page, g_hpage
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(wl, args, world, R)
@@ -380,7 +392,7 @@ def run_ours(args, world, rank, local):
             "l2": f"rotating {R} weight copies ({R * step_bytes / 1e6:.0f} MB, > 3x L2): every step L2-cold",
             "seed": synth.BASE_SEED,
             "body_path": "48 weights in the streaming layout (repacked once at load, same bytes), "
-                         "w4r_matmul_grouped; head: i8_head_logits",
+                         "w4r_matmul_grouped; head in its streaming layout, i8r_head_logits",
             "timing": "a CUDA graph of K steps replayed back to back for about --seconds, CUDA events on the "
                       "replay stream; body_only/head_only (roofline): K launches of that kernel alone per graph, "
                       "replayed the same way",
@@ -391,10 +403,13 @@ def run_ours(args, world, rank, local):
         "body_page_format": {"ms": round(page_avg, 5),
                              "GB_per_s": round(body_bytes() / (page_avg * 1e-3) / 1e9, 1),
                              "kernel": "w4_gemv_kernel<1> (split-K GEMV on the page-format buffers)"},
-        "head_only": {"ms": round(head_avg, 5),
+        "head_only": {"ms": round(head_avg, 5), "kernel": "i8r_head_kernel (streaming layout)",
                       "GB_per_s": round(head_bytes() / (head_avg * 1e-3) / 1e9, 1),
                       "frac_of_hbm": round(head_bytes() / (head_avg * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                      "traffic": profiled_traffic("i8_rows_gpt2_head_m1.md")},
+                      "traffic": profiled_traffic("i8r_head_gpt2_m1.md")},
+        "head_page_format": {"ms": round(hpage_avg, 5),
+                             "GB_per_s": round(head_bytes() / (hpage_avg * 1e-3) / 1e9, 1),
+                             "kernel": "i8_rows_kernel<1> (page-format table)"},
         "frac_of_hbm_step": round(value / n / peaks["hbm_gbs"], 4),
         "roofline": {
             "kernel": "w4r_gemv_m1_kernel (48 repacked weights, one grouped launch)",
@@ -414,6 +429,8 @@ def run_ours(args, world, rank, local):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if world == 1 and not args.no_configs:
+        line["configs"] = run_configs(args, wl, peaks, clocks)
     return line
 
 
@@ -464,6 +481,314 @@ def run_e2e(wl, args, world, R):
     return {"value": round(step_bytes * world / (el / K) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(el / K * 1e3, 5), "tokens_per_s": round(world * K / el, 1)}
+
+
+# ---------------------------------------------------------------- every config
+
+FP32_FMA_PER_SM_CLK = 128  # fp32 FMA lanes per SM per clock (B200)
+
+
+def fp32_alu_peak_tflops(sm_mhz: float | None) -> float:
+    """Dense fp32 FMA peak of the part: SMs x 128 FMA lanes x 2 flops x clock."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    mhz = sm_mhz or 1965.0
+    return sms * FP32_FMA_PER_SM_CLK * 2 * mhz * 1e6 / 1e12
+
+
+def tf32_peak(peaks: dict) -> float:
+    return peaks["bf16_tflops"] * (1.1 / 2.25)  # the nominal dense tf32 : bf16 ratio of the part
+
+
+def graph_ms(calls, reps: int) -> float:
+    """ms per call of `calls` (a list of zero-argument launches, each taking
+    the current stream handle) captured once into a CUDA graph and replayed
+    `reps` times back to back; CUDA events on the replay stream."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        hs = int(side.cuda_stream)
+        with torch.cuda.graph(g, stream=side):
+            for c in calls:
+                c(hs)
+        g.replay()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(side):
+        t0.record(side)
+        for _ in range(reps):
+            g.replay()
+        t1.record(side)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / (reps * len(calls))
+    del g
+    return ms
+
+
+def _ok(st, lib, what):
+    if st != 0:
+        raise RuntimeError(f"{what} failed: {st} {lib.w4_last_error()}")
+
+
+def _oracle_rate(fn, units: float, budget_s: float) -> tuple[float, int, float]:
+    """(units per second, calls, seconds) of the oracle call fn, repeated for about budget_s."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return units * n / el, n, el
+
+
+def _cpu(value, unit, sample, n, el):
+    return {"value": value, "unit": unit, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{sample}: {n} call(s) in {el:.1f} s"}
+
+
+def config0(peaks, budget):
+    """Single W4 768x768, M = 1, repacked, L2-cold (1000 rotating copies)."""
+    import torch
+    import int8_weight_quantized_w4_b200 as w4
+    import oracle
+    K = N = 768
+    W = synth.w4_weight(K, N)
+    dev = torch.device("cuda")
+    qw, sc, zp = (torch.from_numpy(W[k]).to(dev) for k in ("qw", "scales", "zp"))
+    wr0 = w4.w4_repack(qw, sc, zp, K, N)
+    R = max(64, -(-3 * torch.cuda.get_device_properties(0).L2_cache_size // wr0.numel()))
+    wrs = [wr0] + [wr0.clone() for _ in range(R - 1)]
+    x = torch.from_numpy(synth.activations(1, K)).to(dev)
+    y = torch.empty((1, N), device=dev)
+    lib = w4.lib()
+    descs = [w4.make_rdescs([{"x": x, "wr": t, "y": y, "K": K, "N": N}]) for t in wrs]
+    calls = [lambda hs, d=d: _ok(lib.w4r_matmul_grouped(d, 1, hs), lib, "w4r") for d in descs]
+    ms = graph_ms(calls, 10)
+    nbytes = synth.w4_bytes(K, N)
+    xh = synth.activations(1, K)
+    rate, n, el = _oracle_rate(lambda: oracle.w4_matmul_ref(xh, W["qw"], W["scales"], W["zp"], K, N),
+                               nbytes / 1e9, budget)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": "single W4 matmul 768x768, M=1 (streaming layout)", "metric": "weight GB/s",
+            "value": round(gbs, 1), "unit": "GB/s", "us_per_call": round(ms * 1e3, 3),
+            "l2": f"{R} rotating copies ({R * wr0.numel() / 1e6:.0f} MB)",
+            "roofline": {"kernel": "w4r_gemv_m1_kernel", "bound": "hbm", "achieved": round(gbs, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "note": "0.38 MB per call: launch- and latency-bound, reported not targeted"},
+            "cpu_baseline": _cpu(round(rate, 4), "GB/s", "oracle w4_matmul_ref on this weight", n, el)}
+
+
+def config2(peaks, budget):
+    """int8 tied head [768, 50257], last position: M = 1 (streaming layout) and M = 8 (page format)."""
+    import torch
+    import int8_weight_quantized_w4_b200 as w4
+    import oracle
+    K, V = HEAD_K, HEAD_V
+    H = synth.i8_head(K, V)
+    dev = torch.device("cuda")
+    t0_, s0_ = torch.from_numpy(H["table"]).to(dev), torch.from_numpy(H["scales"]).to(dev)
+    tr0 = w4.i8_head_repack(t0_, s0_, K, V)
+    R = max(2, -(-3 * torch.cuda.get_device_properties(0).L2_cache_size // tr0.numel()) + 1)
+    trs = [tr0] + [tr0.clone() for _ in range(R - 1)]
+    tabs = [(t0_, s0_)] + [(t0_.clone(), s0_.clone()) for _ in range(R - 1)]
+    lib = w4.lib()
+    nbytes = synth.i8_head_bytes(K, V)
+    out = {"workload": "int8 tied LM head [768x50257], last position", "l2": f"{R} rotating copies"}
+    h1 = torch.from_numpy(synth.activations(1, K, 999)).to(dev)
+    lg1 = torch.empty((1, V), device=dev)
+    calls = [lambda hs, t=t: _ok(lib.i8r_head_logits(h1.data_ptr(), t.data_ptr(), K, V, lg1.data_ptr(), hs), lib,
+                                 "i8r_head_logits") for t in trs]
+    ms1 = graph_ms(calls, 20)
+    g1 = nbytes / (ms1 * 1e-3) / 1e9
+    M8 = 8
+    h8 = torch.from_numpy(synth.activations(M8, K, 998)).to(dev)
+    lg8 = torch.empty((M8, V), device=dev)
+    wsb = w4.i8_head_workspace_size(M8, K, V)
+    ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)
+    calls8 = [lambda hs, t=t, s=s_: _ok(lib.i8_head_logits(h8.data_ptr(), K, t.data_ptr(), V, s.data_ptr(),
+                                                             lg8.data_ptr(), V, M8, K, V, ws.data_ptr(), ws.numel(),
+                                                             hs), lib, "i8_head_logits")
+              for t, s_ in tabs]
+    ms8 = graph_ms(calls8, 10)
+    g8 = nbytes / (ms8 * 1e-3) / 1e9
+    hh1, hh8 = synth.activations(1, K, 999), synth.activations(M8, K, 998)
+    r1, n1, e1 = _oracle_rate(lambda: oracle.i8_head_ref(hh1, H["table"], H["scales"], K, V), nbytes / 1e9, budget / 2)
+    r8, n8, e8 = _oracle_rate(lambda: oracle.i8_head_ref(hh8, H["table"], H["scales"], K, V), nbytes / 1e9, budget / 2)
+    fl8 = 2 * M8 * K * V / (ms8 * 1e-3) / 1e12
+    out["M1"] = {"metric": "weight GB/s", "value": round(g1, 1), "unit": "GB/s", "us_per_call": round(ms1 * 1e3, 3),
+                 "roofline": {"kernel": "i8r_head_kernel", "bound": "hbm", "achieved": round(g1, 1),
+                              "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(g1 / peaks["hbm_gbs"], 4)},
+                 "cpu_baseline": _cpu(round(r1, 4), "GB/s", "oracle i8_head_ref, M=1", n1, e1)}
+    out["M8"] = {"metric": "weight GB/s", "value": round(g8, 1), "unit": "GB/s", "us_per_call": round(ms8 * 1e3, 3),
+                 "roofline": {"kernel": "i8_head_kernel<8> (page format, stream-K)", "bound": "hbm",
+                              "achieved": round(g8, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": round(g8 / peaks["hbm_gbs"], 4),
+                              "fp32_tflops": round(fl8, 2)},
+                 "cpu_baseline": _cpu(round(r8, 4), "GB/s", "oracle i8_head_ref, M=8", n8, e8)}
+    return out
+
+
+def config3(peaks, budget, wl):
+    """GPT-2 prefill: M = 58 rows through the 48 weights (tensor cores, grouped),
+    then the head on row 57 of the last layer's output (streaming head)."""
+    import torch
+    import int8_weight_quantized_w4_b200 as w4
+    import oracle
+    M = synth.GPT2_PROMPT
+    dev = torch.device("cuda")
+    lib = w4.lib()
+    xs = [torch.from_numpy(synth.activations(M, K, i)).to(dev) for i, (_, K, _) in enumerate(wl.shapes)]
+    ys = [torch.empty((M, N), device=dev) for (_, _, N) in wl.shapes]
+    K, V = HEAD_K, HEAD_V
+    steps = []
+    for r, cp in enumerate(wl.copies):
+        ws = cp[3]
+        descs = w4.make_descs([{"x": xs[i], "y": ys[i], "K": K_, "N": N_, **ws[i]}
+                               for i, (_, K_, N_) in enumerate(wl.shapes)])
+        tr = w4.i8_head_repack(cp[1], cp[2], K, V)
+        steps.append((descs, tr))
+    h = ys[-1][M - 1:M]
+    lg = torch.empty((1, V), device=dev)
+
+    def step(hs, d=None, tr=None):
+        _ok(lib.w4_matmul_grouped(d, len(d), None, 0, hs), lib, "w4_matmul_grouped")
+        _ok(lib.i8r_head_logits(h.data_ptr(), tr.data_ptr(), K, V, lg.data_ptr(), hs), lib, "i8r_head_logits")
+
+    def body_only(hs, d=None):
+        _ok(lib.w4_matmul_grouped(d, len(d), None, 0, hs), lib, "w4_matmul_grouped")
+
+    ms = graph_ms([lambda hs, d=d, tr=tr: step(hs, d, tr) for d, tr in steps], 20)
+    msb = graph_ms([lambda hs, d=d: body_only(hs, d) for d, _ in steps], 20)
+    flops = 2.0 * M * sum(K_ * N_ for _, K_, N_ in wl.shapes)
+    tf = flops / (msb * 1e-3) / 1e12
+    pk = tf32_peak(peaks)
+    W = synth.w4_weight(3072, 768, 3)
+    xh = synth.activations(M, 3072, 3)
+    rate, n, el = _oracle_rate(lambda: oracle.w4_matmul_ref(xh, W["qw"], W["scales"], W["zp"], 3072, 768),
+                               2.0 * M * 3072 * 768 / 1e12, budget)
+    return {"workload": "GPT-2 prefill: M=58 through the 48 W4 weights (tcgen05 3xTF32, grouped) + int8 head "
+                        "on row 57 of the last output (streaming head)",
+            "metric": "prefill TFLOP/s (algorithmic 2MKN, body)", "value": round(tf, 2), "unit": "TFLOP/s",
+            "us_per_step": round(ms * 1e3, 2), "us_body": round(msb * 1e3, 2),
+            "roofline": {"kernel": "w4_tc_kernel (tcgen05.mma kind::tf32, 3 MMAs per product)", "bound": "tensor",
+                         "achieved": round(3 * tf, 2), "achieved_note": "tf32 MMA flops issued: 3x algorithmic",
+                         "peak": round(pk, 1), "unit": "TFLOP/s", "frac": round(3 * tf / pk, 4)},
+            "cpu_baseline": _cpu(round(rate, 6), "TFLOP/s", "oracle w4_matmul_ref, one 3072x768 weight at M=58",
+                                 n, el)}
+
+
+def config4(peaks, budget, clocks):
+    """3.8B-dense-shaped stack, 32 layers x [3072x9216, 3072x3072, 3072x16384,
+    8192x3072]: decode at M = 1 (streaming layout), 8 (split-K GEMV) and 32
+    (tensor cores), prefill at M = 2048 (tensor cores). 128 distinct weights
+    (2.32 GB: L2-cold by size), generated on the GPU with a seeded generator
+    in the synthetic distributions (uniform nibbles, scales U[0.005, 0.02])."""
+    import torch
+    import int8_weight_quantized_w4_b200 as w4
+    import oracle
+    dev = torch.device("cuda")
+    lib = w4.lib()
+    shapes = [(K, N) for _, K, N in synth.dense38_stack_shapes()]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(synth.BASE_SEED + 38)
+    weights = []
+    for K, N in shapes:
+        nb = K // 32
+        qw = torch.randint(0, 256, (K * N // 2,), dtype=torch.uint8, device=dev, generator=gen)
+        sc = torch.empty((nb, N), device=dev).uniform_(0.005, 0.02, generator=gen)
+        zp = torch.randint(0, 256, (nb * N // 2,), dtype=torch.uint8, device=dev, generator=gen)
+        weights.append({"qw": qw, "scales": sc, "zp": zp})
+    nbytes = sum(synth.w4_bytes(K, N) for K, N in shapes)
+    wsum = sum(K * N for K, N in shapes)
+    out = {"workload": "3.8B-dense-shaped W4 stack: 32 layers x [3072x9216, 3072x3072, 3072x16384, 8192x3072], "
+                       "128 distinct weights", "weight_bytes": nbytes}
+    # decode M = 1 on the streaming layout
+    wrs = [w4.w4_repack(Wd["qw"], Wd["scales"], Wd["zp"], K, N) for Wd, (K, N) in zip(weights, shapes)]
+    x1 = {K: torch.randn((1, K), device=dev, generator=gen) for K in (3072, 8192)}
+    y1 = [torch.empty((1, N), device=dev) for _, N in shapes]
+    rd = w4.make_rdescs([{"x": x1[K], "wr": wrs[i], "y": y1[i], "K": K, "N": N} for i, (K, N) in enumerate(shapes)])
+    ms1 = graph_ms([lambda hs: _ok(lib.w4r_matmul_grouped(rd, len(rd), hs), lib, "w4r")], 20)
+    del wrs
+    g1 = nbytes / (ms1 * 1e-3) / 1e9
+    out["decode_M1"] = {"metric": "weight GB/s", "value": round(g1, 1), "unit": "GB/s",
+                        "ms_per_step": round(ms1, 4), "tokens_per_s": round(1e3 / ms1, 1),
+                        "roofline": {"kernel": "w4r_gemv_m1_kernel", "bound": "hbm", "achieved": round(g1, 1),
+                                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": round(g1 / peaks["hbm_gbs"], 4)}}
+    # decode M = 8 (split-K GEMV) and M = 32 (tensor cores), page format
+    for M in (8, 32):
+        xm = {K: torch.randn((M, K), device=dev, generator=gen) for K in (3072, 8192)}
+        ym = [torch.empty((M, N), device=dev) for _, N in shapes]
+        items = [{"x": xm[K], "y": ym[i], "K": K, "N": N, **weights[i]} for i, (K, N) in enumerate(shapes)]
+        descs = w4.make_descs(items)
+        wsb = w4.w4_matmul_grouped_workspace_size(descs)
+        ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)
+        msm = graph_ms([lambda hs: _ok(lib.w4_matmul_grouped(descs, len(descs), ws.data_ptr(), ws.numel(), hs), lib,
+                                       "w4_matmul_grouped")], 5)
+        tfl = 2.0 * M * wsum / (msm * 1e-3) / 1e12
+        gb = nbytes / (msm * 1e-3) / 1e9
+        if M == 8:
+            pk = fp32_alu_peak_tflops(clocks.get("sm_mhz"))
+            roof = {"kernel": "w4_gemv_kernel<8> (split-K GEMV)", "bound": "alu", "achieved": round(tfl, 2),
+                    "peak": round(pk, 1), "unit": "TFLOP/s", "frac": round(tfl / pk, 4),
+                    "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x the sampled SM clock"}
+        else:
+            pk = tf32_peak(peaks)
+            roof = {"kernel": "w4_tc_kernel (3xTF32)", "bound": "tensor", "achieved": round(3 * tfl, 2),
+                    "achieved_note": "tf32 MMA flops issued: 3x algorithmic", "peak": round(pk, 1),
+                    "unit": "TFLOP/s", "frac": round(3 * tfl / pk, 4)}
+        out[f"decode_M{M}"] = {"metric": "TFLOP/s (algorithmic 2MKN)", "value": round(tfl, 2), "unit": "TFLOP/s",
+                               "weight_GB_per_s": round(gb, 1), "ms_per_step": round(msm, 4), "roofline": roof}
+        del xm, ym, items, descs, ws
+    # prefill M = 2048 (tensor cores): x shared by the weights of one K, y distinct per weight
+    M = 2048
+    xp = {K: torch.randn((M, K), device=dev, generator=gen) for K in (3072, 8192)}
+    yp = [torch.empty((M, N), device=dev) for _, N in shapes]
+    descs = w4.make_descs([{"x": xp[K], "y": yp[i], "K": K, "N": N, **weights[i]} for i, (K, N) in enumerate(shapes)])
+    msp = graph_ms([lambda hs: _ok(lib.w4_matmul_grouped(descs, len(descs), None, 0, hs), lib, "w4_matmul_grouped")], 2)
+    tfp = 2.0 * M * wsum / (msp * 1e-3) / 1e12
+    pk = tf32_peak(peaks)
+    out["prefill_M2048"] = {"metric": "prefill TFLOP/s (algorithmic 2MKN)", "value": round(tfp, 2), "unit": "TFLOP/s",
+                            "ms_per_step": round(msp, 3),
+                            "roofline": {"kernel": "w4_tc_kernel (tcgen05.mma kind::tf32, 3 MMAs per product)",
+                                         "bound": "tensor", "achieved": round(3 * tfp, 1),
+                                         "achieved_note": "tf32 MMA flops issued: 3x algorithmic",
+                                         "peak": round(pk, 1), "unit": "TFLOP/s", "frac": round(3 * tfp / pk, 4),
+                                         "frac_algorithmic": round(tfp / pk, 4)}}
+    del xp, yp, descs, weights
+    torch.cuda.empty_cache()
+    # the oracle on one o_proj weight (3072x3072) at each M, scaled to the metric
+    W = synth.w4_weight(3072, 3072, 38)
+    per = {}
+    for M, key, unit in ((1, "decode_M1", "GB/s"), (8, "decode_M8", "TFLOP/s"), (32, "decode_M32", "TFLOP/s"),
+                         (2048, "prefill_M2048", "TFLOP/s")):
+        xh = synth.activations(M, 3072, 38)
+        units = synth.w4_bytes(3072, 3072) / 1e9 if unit == "GB/s" else 2.0 * M * 3072 * 3072 / 1e12
+        r, n, el = _oracle_rate(lambda: oracle.w4_matmul_ref(xh, W["qw"], W["scales"], W["zp"], 3072, 3072), units,
+                                budget / 4)
+        out[key]["cpu_baseline"] = _cpu(round(r, 6), unit, f"oracle w4_matmul_ref, one 3072x3072 weight at M={M}",
+                                        n, el)
+    return out
+
+
+def run_configs(args, wl, peaks, clocks) -> dict:
+    """Every workload the decode step does not cover, each with its roofline
+    and a bounded oracle sample (N = 1 only)."""
+    res = {}
+    budget = args.cpu_seconds / 4
+    for name, fn in (("config0", lambda: config0(peaks, budget)), ("config2", lambda: config2(peaks, budget)),
+                     ("config3", lambda: config3(peaks, budget, wl)), ("config4", lambda: config4(peaks, budget, clocks))):
+        t0 = time.perf_counter()
+        try:
+            res[name] = fn()
+        except Exception as e:  # one config failing must not lose the headline line
+            res[name] = {"error": f"{type(e).__name__}: {e}"}
+        res[name]["wall_s"] = round(time.perf_counter() - t0, 1)
+    return res
 
 
 # ---------------------------------------------------------------- oracle on the host
@@ -685,6 +1010,7 @@ def main():
     ap.add_argument("--seconds", type=float, default=1.0,
                     help="device seconds of the timed step replays (the body and head alone get half each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-config measurements (configs 0, 2, 3, 4)")
     ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
                     help="decode: the GPT-2 decode step (the headline); prefill: the 3.8B-shaped stack at M=2048")
     args = ap.parse_args()
