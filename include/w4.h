@@ -270,6 +270,57 @@ typedef struct w4r_desc {
 W4_API w4_status w4r_matmul_grouped(const w4r_desc* descs, int32_t count, void* stream);
 W4_API w4_status w4r_matmul(const w4r_desc* d, void* stream);
 
+/* ------------------------------------------------------------------ tile layout (prefill) */
+
+/* The tile layout of one W4 weight, read by the tensor-core tile GEMM: the
+ * page-format nibbles, scales and zero points ("ONNX export, quantization and
+ * the browser runtime", section "Quantization (train/quantize.py)", step 2)
+ * reordered once at load time, nothing rounded (w4t_repack_restore gives the
+ * page buffers back bit for bit). K % 32 == 0, N % 8 == 0, K <= 2^24,
+ * N <= 2^23; tiles of 128 columns (the last padded with zero weights) in
+ * column order, each K / 32 blocks of 2624 bytes:
+ *   block b of tile T: [0, 2048) column c (0..127) at c * 16, four words;
+ *     word j holds rows 32 b + 8 j + r (r = 0..7) of column 128 T + c with
+ *     row r in bits {0-3, 16-19, 4-7, 20-23, 8-11, 24-27, 12-15, 28-31}[r];
+ *   [2048, 2560) the block's scales, column c at 2048 + 4 c;
+ *   [2560, 2624) its zero points packed as the page packs them (word w:
+ *     columns 8 w .. 8 w + 7, nibble i = column 8 w + i).
+ * w4t_repacked_bytes() is the size (the page-format total when N % 128 == 0;
+ * 0 for a shape the layout does not take). Repack and restore: as
+ * w4_repack / w4_repack_restore (device buffers, 16-byte aligned,
+ * asynchronous). */
+W4_API size_t w4t_repacked_bytes(int64_t K, int64_t N);
+W4_API w4_status w4t_repack(const uint8_t* qw, const float* scales, const uint8_t* zp, int64_t K, int64_t N,
+                            void* wt, void* stream);
+W4_API w4_status w4t_repack_restore(const void* wt, int64_t K, int64_t N, uint8_t* qw, float* scales, uint8_t* zp,
+                                    void* stream);
+
+/* Matmuls y = act(x . W + bias) + residual on weights in the tile layout, for
+ * any M (built for prefill, M > 16), on the tensor cores. Per K-block the
+ * weights' (q - zp) are exact in bf16; each x is split exactly into three
+ * bf16 pieces (x = p0 + p1 + p2, 8 + 8 + 8 significant bits), so every
+ * product is exact; tcgen05.mma sums a block's products in fp32 and the
+ * block's scale is applied in fp32 (y += s * sum). Non-finite x give NaN.
+ * - descs: HOST array of w4t_desc (the w4r_desc fields; wr = the tile-layout
+ *   weight), read during the call only. Any M >= 0 up to 131072, K % 32 == 0,
+ *   N % 8 == 0, ldx >= K, ldy >= N, ldr >= N when residual is set; x / y /
+ *   bias / residual 4-byte aligned, wr 16-byte aligned. K = 0 writes the
+ *   epilogue of 0. Outputs must not overlap each other or any input.
+ * - workspace: device memory of at least w4t_workspace_size(descs, count)
+ *   bytes, 16-byte aligned (NULL when that is 0); it receives the pieces of
+ *   each distinct x (same x pointer, ldx, M and K share them) and needs no
+ *   zeroing. Calls that may run at the same time must not share it.
+ * - The pieces are written by one launch, then the tile GEMM runs (a second
+ *   launch per class of rows-per-tile: 16, 32, 64 or 128 by M); both start
+ *   early on the stream (programmatic dependent launch) and read x, bias and
+ *   the residual and write y only after the previous work on the stream has
+ *   completed. */
+typedef w4r_desc w4t_desc;
+W4_API size_t w4t_workspace_size(const w4t_desc* descs, int32_t count);
+W4_API w4_status w4t_matmul_grouped(const w4t_desc* descs, int32_t count, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+W4_API w4_status w4t_matmul(const w4t_desc* d, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------ head */
 
 /* Bytes of workspace i8_head_logits needs for this shape on the current

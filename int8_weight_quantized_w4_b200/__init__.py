@@ -218,7 +218,7 @@ def make_rdescs(items: Sequence[dict]):
         K, N = int(it["K"]), int(it["N"])
         M = x.shape[0] if x.dim() == 2 else 1
         b, r, ldr, a = _epilogue(it, N)
-        arr[i] = W4RDesc(_ptr(x), K, _ptr(it["wr"]), _ptr(y), N, M, K, N, b, r, ldr, a, 0)
+        arr[i] = W4RDesc(_ptr(x), _ld(x, K), _ptr(it["wr"]), _ptr(y), _ld(y, N), M, K, N, b, r, ldr, a, 0)
     return arr
 
 
@@ -237,6 +237,86 @@ def w4r_matmul(x, wr, K: int, N: int, y=None, stream=None, bias=None, residual=N
         y = torch.empty((1, N), dtype=torch.float32, device=x.device)
     item = {"x": x, "wr": wr, "y": y, "K": K, "N": N, "bias": bias, "residual": residual, "act": act}
     w4r_matmul_grouped(descs=make_rdescs([item]), stream=stream)
+    return y
+
+
+# ---------------------------------------------------------------- tile layout (prefill)
+
+_TWS: dict = {}
+
+
+def tile_workspace(nbytes: int, device=None):
+    """A device scratch of at least nbytes for w4t_matmul_grouped (cached per
+    device; no zeroing needed). Calls that may overlap on the GPU must not
+    share one: pass your own."""
+    torch = _torch()
+    if nbytes == 0:
+        return None
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    idx = dev.index if dev.index is not None else torch.cuda.current_device()
+    cur = _TWS.get(idx)
+    if cur is None or cur.numel() < nbytes:
+        cur = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=dev)
+        _TWS[idx] = cur
+    return cur
+
+
+def w4t_repacked_bytes(K: int, N: int) -> int:
+    return int(lib().w4t_repacked_bytes(K, N))
+
+
+def w4t_repack(qw, scales, zp, K: int, N: int, out=None, stream=None):
+    """The weight (page format) in the tile layout the tensor-core tile GEMM
+    reads: a uint8 device tensor of w4t_repacked_bytes(K, N) bytes."""
+    torch = _torch()
+    nbytes = w4t_repacked_bytes(K, N)
+    if nbytes == 0:
+        raise ValueError(f"the tile layout does not take K={K}, N={N} (K % 32 == 0, N % 8 == 0)")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=qw.device)
+    _check(lib().w4t_repack(_ptr(qw), _ptr(scales), _ptr(zp), K, N, _ptr(out), _stream_handle(stream)), "w4t_repack")
+    return out
+
+
+def w4t_repack_restore(wt, K: int, N: int, stream=None):
+    """The page-format buffers (qw, scales, zp) of a weight in the tile layout."""
+    torch = _torch()
+    nb = K // 32
+    qw = torch.empty(K * N // 2, dtype=torch.uint8, device=wt.device)
+    sc = torch.empty((nb, N), dtype=torch.float32, device=wt.device)
+    zp = torch.empty(nb * N // 2, dtype=torch.uint8, device=wt.device)
+    _check(lib().w4t_repack_restore(_ptr(wt), K, N, _ptr(qw), _ptr(sc), _ptr(zp), _stream_handle(stream)),
+           "w4t_repack_restore")
+    return qw, sc, zp
+
+
+def w4t_workspace_size(descs) -> int:
+    return int(lib().w4t_workspace_size(descs, len(descs)))
+
+
+def w4t_matmul_grouped(items: Sequence[dict] | None = None, descs=None, ws=None, stream=None):
+    """Matmuls of any M on tile-layout weights ("wr" = w4t_repack output) on
+    the tensor cores; items as for make_rdescs (x [M, K])."""
+    if descs is None:
+        descs = make_rdescs(items)
+    need = w4t_workspace_size(descs)
+    if ws is None:
+        ws = tile_workspace(need)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().w4t_matmul_grouped(descs, len(descs), _ptr(ws), nbytes, _stream_handle(stream)),
+           "w4t_matmul_grouped")
+
+
+def w4t_matmul(x, wt, K: int, N: int, y=None, ws=None, stream=None, bias=None, residual=None, act: str = "none"):
+    """y[M, N] = act(x[M, K] . W + bias) + residual with W in the tile layout
+    (w4t_repack); returns y."""
+    torch = _torch()
+    if x.dim() == 1:
+        x = x.view(1, -1)
+    if y is None:
+        y = torch.empty((x.shape[0], N), dtype=torch.float32, device=x.device)
+    item = {"x": x, "wr": wt, "y": y, "K": K, "N": N, "bias": bias, "residual": residual, "act": act}
+    w4t_matmul_grouped(descs=make_rdescs([item]), ws=ws, stream=stream)
     return y
 
 

@@ -87,6 +87,13 @@ SIGNATURES = {
     "w4_repack_restore": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p,
                                     C.c_void_p]),
     "w4r_matmul": (C.c_int, [C.POINTER(W4RDesc), C.c_void_p]),
+    "w4t_repacked_bytes": (C.c_size_t, [C.c_int64, C.c_int64]),
+    "w4t_repack": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),
+    "w4t_repack_restore": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p,
+                                     C.c_void_p]),
+    "w4t_workspace_size": (C.c_size_t, [C.POINTER(W4RDesc), C.c_int32]),
+    "w4t_matmul_grouped": (C.c_int, [C.POINTER(W4RDesc), C.c_int32, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "w4t_matmul": (C.c_int, [C.POINTER(W4RDesc), C.c_void_p, C.c_size_t, C.c_void_p]),
     "w4r_matmul_grouped": (C.c_int, [C.POINTER(W4RDesc), C.c_int32, C.c_void_p]),
     "i8_head_repacked_bytes": (C.c_size_t, [C.c_int64, C.c_int64]),
     "i8_head_repack": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),

@@ -1,0 +1,1171 @@
+// w4t: y = x . W for many rows of x (prefill) on the 5th-generation tensor
+// cores, with W4 weights in their tile layout.
+//
+// The weight format is the one of "ONNX export, quantization and the browser
+// runtime", section "Quantization (train/quantize.py)", step 2 (dq4): blocks
+// of 32 along K, one fp32 scale and one uint4 zero point per (block,
+// column), w = (q - zp) * scale; y = x . W with fp32 compute.
+//
+// Tile layout (K % 32 == 0, N % 8 == 0): tiles of 128 columns (the last one
+// padded with zero weights), each all K rows, in column order; a tile is
+// K / 32 blocks of 2624 bytes, one per K-block b:
+//   [0, 2048)    column c (0..127) at c * 16: four words, word j holding rows
+//                32 b + 8 j + r (r = 0..7) with row r in bits
+//                {0-3, 16-19, 4-7, 20-23, 8-11, 24-27, 12-15, 28-31}[r]
+//   [2048, 2560) the block's scales, column c at 2048 + 4 c
+//   [2560, 2624) the block's zero points, the page's packing: word w holds
+//                columns 8 w .. 8 w + 7 (nibble i = column 8 w + i)
+// Every nibble, scale and zero point of the page format is there once;
+// restoring gives the page-format buffers back bit for bit.
+//
+// Arithmetic. Per block b and column n,
+//   sum_{k in b} x_k w_kn = s_bn * sum_{k in b} x_k (q_kn - zp_bn).
+// q - zp is an integer in [-15, 15], exact in bf16. Each x_k is split exactly
+// into three bf16 pieces, x = p0 + p1 + p2 (p0 is x with the low 16 bits
+// cleared, p1 the same of x - p0, p2 the rest: 8 + 8 + 8 significant bits),
+// so every product p_i (q - zp) is exact. The tensor core sums the products
+// of a block in fp32 (two K-steps x three pieces = six MMAs into a fresh
+// accumulator) and the block's scale is applied once per column and row in
+// fp32: y += s * D.
+//
+// Design (sm_100a):
+//  * w4t_split_kernel writes the pieces of each x once per call into the
+//    caller's workspace, already in the MMA's shared-memory operand layout
+//    (K-major, no swizzle: core matrices of 8 rows x 16 bytes, the two 8-wide
+//    K halves of a K-step 128 bytes apart, groups of 8 rows 256 bytes
+//    apart). Rows come in tiles of NX = 16, 32, 64 or 128 (by M); one block
+//    of one row tile is one contiguous run of 192 NX bytes: piece p, K-step h
+//    at p * 64 NX + h * 32 NX. Rows past M are zeros.
+//  * w4t_gemm_kernel: one persistent CTA per SM over a list of (row tile,
+//    128-column tile) pairs that the host deals out largest first. The MMA's
+//    M = 128 are the weight's columns (operand A, in tensor memory: decoded
+//    in registers, no shared-memory round trip), its N = NX are x's rows
+//    (operand B, in shared memory); the accumulator D[column][row] is in
+//    tensor memory, one per block in flight (3 to 8 blocks, by NX).
+//    - warp 0 streams each block's pieces and weight bytes (one bulk copy
+//      each, no multicast) through a ring of stages;
+//    - warps 1 and 2 take the blocks in turn and issue a block's six MMAs
+//      (kind::f16, M 128, N NX, K 16) once the decode warps report it ready
+//      (bytes landed, A decoded, accumulator free), then commit them to the
+//      accumulator's barrier. The issuing thread waits on one barrier and
+//      commits once per block: its barrier operations slow the MMAs it has
+//      in flight. Two issuers: one waits while the other is held in issue;
+//    - warps 3..10 (two per quarter of tensor-memory lanes, taking the
+//      blocks in turn; a thread owns one column of the tile) turn a block's
+//      nibbles into bf16 (q - zp) with one LOP3 and one bf16x2 subtraction
+//      per pair and store them with tcgen05.st, up to NSLOT - 1 blocks ahead
+//      of the tensor core;
+//    - warps 11..18 (two per quarter, each half of the accumulator columns)
+//      read each block's accumulator back (tcgen05.ld) and add s * D to
+//      registers; after a tile's last block they apply the fused epilogue
+//      and store y, each warp 32 consecutive columns of a row at a time.
+//  * Every wait is bounded; on timeout the CTA records the error, stops
+//    issuing work, lets its copies and MMAs in flight finish, and returns.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <memory>
+#include <queue>
+#include <vector>
+
+#include "w4_device.cuh"
+#include "w4_internal.h"
+
+namespace {
+
+using namespace w4dev;
+
+constexpr int TN = 128;           // columns of a tile = MMA M
+constexpr int BLK = 2624;         // bytes of one block of a tile
+// Warps: producer, 2 MMA issuers, decode warps (one or two per quarter of
+// tensor-memory lanes), read-back warps (two or four per quarter, 32
+// accumulators each). Decode costs the same per block whatever NX is, so
+// 128-row tiles (twice the MMA work per block) need one decode warp per
+// quarter, and four read-back warps per quarter to hold their 128 rows.
+__host__ __device__ constexpr int decode_warps(int nx) { return nx >= 128 ? 4 : 8; }
+__host__ __device__ constexpr int readback_warps(int nx) { return nx >= 128 ? 16 : 8; }
+__host__ __device__ constexpr int block_threads(int nx) { return (3 + decode_warps(nx) + readback_warps(nx)) * 32; }
+constexpr int TCAP = 48;          // matrices per launch
+constexpr int LCAP = 4096;        // tile-list entries per launch
+constexpr int RING = 196608;      // bytes of the stage ring
+constexpr int MAXST = 16;         // stages at most
+constexpr int MAXSLOT = 8;        // blocks in flight between decode and read-back, at most
+constexpr uint32_t TCOLS = 512;   // tensor memory: per slot NX accumulator columns (from 0) and 16 A columns
+constexpr int OFF_BAR = RING;
+constexpr int SMEM_BYTES = OFF_BAR + (2 * MAXST + 3 * MAXSLOT) * 8 + 16;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
+
+// bytes of one block of one row tile of pieces, and of one stage
+__host__ __device__ constexpr int piece_bytes(int nx) { return 192 * nx; }
+__host__ __device__ constexpr int stage_bytes(int nx) { return (192 * nx + BLK + 127) / 128 * 128; }
+__host__ __device__ constexpr int ring_stages(int nx) {
+  return RING / stage_bytes(nx) < MAXST ? RING / stage_bytes(nx) : MAXST;
+}
+// Slots of tensor memory (an accumulator of NX columns and an A operand of
+// 16): as many as 512 columns hold, at most MAXSLOT (3 for NX = 128, 6 for 64,
+// 8 below). A block's slot is busy from its decode to its read-back, so more
+// slots keep more blocks between the two.
+__host__ __device__ constexpr int tmem_slots(int nx) {
+  return static_cast<int>(TCOLS) / (nx + 16) < MAXSLOT ? static_cast<int>(TCOLS) / (nx + 16) : MAXSLOT;
+}
+
+struct TMat {
+  const uint8_t* wt;  // tile layout
+  const uint8_t* xp;  // pieces of x (workspace)
+  float* y;
+  const float* bias;
+  const float* res;
+  int64_t ldy, ldr;
+  int32_t M, N, nb, act;
+};
+
+struct TParams {
+  TMat m[TCAP];
+  uint32_t first[257];  // CTA c takes list[first[c] .. first[c + 1])
+  uint32_t list[LCAP];  // (matrix << 26) | (row tile << 16) | column tile
+  ErrorWord* err;
+  uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Bounded wait that ignores the abort flag: used only to let work already in
+// flight (copies, MMAs) land before the CTA returns.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
+  while (!mbar_try_wait_sleep(a, parity, 100000u))
+    if (globaltimer_ns() - t0 > timeout_ns) return;
+}
+
+// K-major, no swizzle, LBO 128 bytes, SBO 256 bytes, version 1.
+__device__ __forceinline__ uint64_t bdesc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((128u >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((256u >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// D (tensor memory) (+)= A (tensor memory) . B (shared memory), kind::f16
+// with bf16 operands and an fp32 accumulator.
+__device__ __forceinline__ void mma_bf16(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, bool acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(acc ? 1u : 0u)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// bf16x2 {128 + q_lo, 128 + q_hi} from the nibbles in bits 0-3 and 16-19
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(w));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&a)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "r"(a[8]), "r"(a[9]),
+      "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]), "r"(a[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+
+// R consecutive accumulator columns of this thread's lane (R = 8 .. 64)
+template <int R>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[R]) {
+  if constexpr (R == 8) {
+    tmem_ld8(taddr, v);
+  } else if constexpr (R == 16) {
+    tmem_ld16(taddr, v);
+  } else {
+#pragma unroll
+    for (int i = 0; i < R / 32; ++i) tmem_ld32(taddr + 32 * i, v + 32 * i);
+  }
+}
+
+// One CTA's walk over its (tile, block) sequence.
+struct Walk {
+  int t, b;           // tile ordinal in the CTA's list, block in the tile
+  int g, xt, ct, nb;  // the tile: matrix, row tile, column tile, blocks
+};
+
+__device__ __forceinline__ void walk_load(Walk& w, const TParams& p, uint32_t first) {
+  const uint32_t e = p.list[first + w.t];
+  w.g = static_cast<int>(e >> 26);
+  w.xt = static_cast<int>((e >> 16) & 1023u);
+  w.ct = static_cast<int>(e & 0xFFFFu);
+  w.nb = p.m[w.g].nb;
+}
+
+// The K-block read at step b of a tile. The column tiles of one row tile
+// read the same x pieces; each starts at its own block (5 ct mod nb) so that
+// the SMs streaming them at the same time read different bytes instead of
+// all asking L2 for the same lines. Every step reads a different block.
+__device__ __forceinline__ int kblock(const Walk& w) {
+  int k = w.b + (w.ct * 5) % w.nb;
+  return k >= w.nb ? k - w.nb : k;
+}
+
+__device__ __forceinline__ bool walk_next(Walk& w, const TParams& p, uint32_t first, int ntl) {
+  if (++w.b < w.nb) return true;
+  w.b = 0;
+  if (++w.t >= ntl) return false;
+  walk_load(w, p, first);
+  return true;
+}
+
+template <int NX>
+__global__ void __launch_bounds__(block_threads(NX), 1) w4t_gemm_kernel(const __grid_constant__ TParams p) {
+  constexpr int PB = piece_bytes(NX);
+  constexpr int SB = stage_bytes(NX);
+  constexpr int NST = ring_stages(NX);
+  constexpr int NSLOT = tmem_slots(NX);
+  constexpr uint32_t ACOL = static_cast<uint32_t>(NSLOT * NX);  // A slots after the accumulators
+  constexpr int NDEC = decode_warps(NX);
+  constexpr int NRB = readback_warps(NX);
+  constexpr int RB0 = 3 + NDEC;         // first read-back warp
+  constexpr int HR = NX / (NRB / 4);    // accumulator columns (rows of x) per read-back warp
+  constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(NX) >> 3) << 17) |
+                             ((static_cast<uint32_t>(TN) >> 4) << 24);
+  static_assert(NST >= 2, "at least two stages");
+
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t first = p.first[blockIdx.x];
+  const int ntl = static_cast<int>(p.first[blockIdx.x + 1] - first);
+
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + MAXST;
+  uint64_t* aready = empty + MAXST;     // [NSLOT]: the block ready for its MMAs
+  uint64_t* dready = aready + MAXSLOT;  // [NSLOT]: the block's MMAs done
+  uint64_t* dfree = dready + MAXSLOT;   // [NSLOT]: accumulator read back
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(dfree + MAXSLOT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                 "r"(TCOLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4 + NRB);  // the block's 4 decode warps and the read-back warps (after its MMAs)
+    }
+    for (int i = 0; i < NSLOT; ++i) {
+      mbar_init(&aready[i], 4);
+      mbar_init(&dready[i], 1);
+      mbar_init(&dfree[i], NRB);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && ntl > 0) {
+      pdl_wait();  // the pieces are the split kernel's output
+      Walk w{0, 0, 0, 0, 0, 0};
+      walk_load(w, p, first);
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      // the tile's first block (staggered start) and its source addresses
+      const uint8_t* xsrc = nullptr;
+      const uint8_t* wsrc = nullptr;
+      int blk = 0;
+      auto tile_start = [&]() {
+        const TMat& m = p.m[w.g];
+        blk = kblock(w);
+        xsrc = m.xp + (static_cast<int64_t>(w.xt) * m.nb) * PB;
+        wsrc = m.wt + (static_cast<int64_t>(w.ct) * m.nb) * BLK;
+      };
+      tile_start();
+#pragma unroll 1
+      while (true) {
+        if (issued >= NST && !mbar_wait_bounded(&empty[s], ph ^ 1u, p.timeout_ns, abort_flag, p.err, K_TILE, 1)) break;
+        uint8_t* st = smem + s * SB;
+        mbar_arrive_expect_tx(&full[s], PB + BLK);
+        bulk_g2s(st, xsrc + static_cast<int64_t>(blk) * PB, PB, &full[s]);
+        bulk_g2s(st + PB, wsrc + static_cast<int64_t>(blk) * BLK, BLK, &full[s]);
+        ++issued;
+        if (++s == NST) {
+          s = 0;
+          ph ^= 1u;
+        }
+        if (++blk == w.nb) blk = 0;
+        if (++w.b == w.nb) {
+          w.b = 0;
+          if (++w.t >= ntl) break;
+          walk_load(w, p, first);
+          tile_start();
+        }
+      }
+      // copies in flight land before the CTA may return
+      for (int i = issued > NST ? issued - NST : 0; i < issued; ++i)
+        mbar_wait_drain(&full[i % NST], static_cast<uint32_t>(i / NST) & 1u, p.timeout_ns);
+    }
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two warps take the blocks in turn (even / odd): while one is held in
+    // tcgen05.mma issue (the tensor core takes an MMA when it can start it),
+    // the other checks its next block's barriers, so the tensor core sees
+    // no gap between blocks.
+    const int par = warp - 1;
+    if (lane == 0 && ntl > 0) {
+      // the CTA's blocks in all; this issuer's are par, par + 2, ...; the
+      // stage and slot of a block follow from its number alone
+      int J = 0;
+      for (int t = 0; t < ntl; ++t) J += p.m[p.list[first + t] >> 26].nb;
+      int j = par, s = par % NST, d = par % NSLOT;
+      uint32_t dph = 0;
+      const uint64_t desc0 = bdesc(smem_u32(smem));
+      const long long budget = static_cast<long long>(p.timeout_ns) * 2;  // clocks, at most 2 per ns
+#pragma unroll 1
+      while (j < J) {
+        // aready(j) stands for the whole block: the decode warps saw its
+        // bytes land (full) and its slot read back (dfree) before they
+        // arrived on it. Spin on it with plain try_wait: the issuing thread
+        // is the tensor core's only feed, so it must resume at once.
+        const uint32_t ab = smem_u32(&aready[d]);
+        if (!mbar_try_wait(ab, dph)) {
+          const long long t0 = clock64();
+          bool ok = false;
+#pragma unroll 1
+          for (uint32_t it = 1;; ++it) {
+            if (mbar_try_wait(ab, dph)) {
+              ok = true;
+              break;
+            }
+            if ((it & 63u) == 0 && (*abort_flag || clock64() - t0 > budget)) break;
+          }
+          if (!ok) {
+            if (!*abort_flag) {
+              *abort_flag = 1;
+              record_error(p.err, W4_ERR_TIMEOUT, K_TILE, 3);
+            }
+            break;
+          }
+        }
+        tc_fence_after();
+        const uint32_t dt = tmem + static_cast<uint32_t>(d * NX);
+        const uint32_t at = tmem + ACOL + static_cast<uint32_t>(d * 16);
+        const uint64_t ds = desc0 + static_cast<uint64_t>(s * (SB >> 4));  // B slabs, 16-byte units
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int pc = 0; pc < 3; ++pc)
+            mma_bf16(dt, at + 8 * h, ds + static_cast<uint64_t>((pc * 64 * NX + h * 32 * NX) >> 4), IDESC, (h | pc) != 0);
+        mma_commit(&dready[d]);
+        j += 2;
+        s += 2;
+        if (s >= NST) s -= NST;
+        d += 2;
+        if (d >= NSLOT) {
+          d -= NSLOT;
+          dph ^= 1u;
+        }
+      }
+      // this issuer's last commit covers every MMA it issued
+      const int last = j - 2;
+      if (last >= 0 && last < J)
+        mbar_wait_drain(&dready[last % NSLOT], static_cast<uint32_t>(last / NSLOT) & 1u, p.timeout_ns);
+    }
+  } else if (warp < RB0) {
+    // ------------------------------------------------------------ decode
+    // Warps 3..10, two per quarter of tensor-memory lanes (a thread owns one
+    // column of the tile), taking the blocks in turn (warps 3..6 the even
+    // ones, 7..10 the odd ones): block j goes into slot j % NSLOT once block
+    // j - NSLOT, the slot's last user, has been read back (its MMAs are then
+    // done and its accumulator free).
+    const int q = warp & 3;
+    const int par = NDEC == 8 ? (warp - 3) >> 2 : -1;  // with 4 decode warps each takes every block
+    const int c = 32 * q + lane;
+    const uint32_t lanes = static_cast<uint32_t>(32 * q) << 16;
+    Walk w{0, 0, 0, 0, 0, 0};
+    bool more = ntl > 0;
+    if (more) walk_load(w, p, first);
+    int s = 0, d = 0, j = 0;
+    uint32_t ph = 0, dph = 0;
+#pragma unroll 1
+    while (more) {
+      if (par >= 0 && (j & 1) != par) {  // the other warp of the quarter decodes this block
+        ++j;
+        if (++s == NST) {
+          s = 0;
+          ph ^= 1u;
+        }
+        if (++d == NSLOT) {
+          d = 0;
+          dph ^= 1u;
+        }
+        more = walk_next(w, p, first, ntl);
+        continue;
+      }
+      bool okw = mbar_wait_bounded(&full[s], ph, p.timeout_ns, abort_flag, p.err, K_TILE, 5);
+      if (okw && j >= NSLOT) okw = mbar_wait_bounded(&dfree[d], dph ^ 1u, p.timeout_ns, abort_flag, p.err, K_TILE, 7);
+      if (!__all_sync(0xffffffffu, okw)) break;
+      tc_fence_after();
+      const uint8_t* wb = smem + s * SB + PB;
+      const uint4 wv = *reinterpret_cast<const uint4*>(wb + c * 16);
+      const uint32_t zw = *reinterpret_cast<const uint32_t*>(wb + 2560 + (c >> 3) * 4);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      const uint32_t z = (zw >> (4 * (c & 7))) & 0xFu;
+      const uint32_t zc = 0x43004300u | z | (z << 16);  // bf16x2 {128 + zp, 128 + zp}
+      uint32_t a[16];
+      const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        a[4 * k + 0] = bf16x2_sub(nib_pair(ws[k]), zc);
+        a[4 * k + 1] = bf16x2_sub(nib_pair(ws[k] >> 4), zc);
+        a[4 * k + 2] = bf16x2_sub(nib_pair(ws[k] >> 8), zc);
+        a[4 * k + 3] = bf16x2_sub(nib_pair(ws[k] >> 12), zc);
+      }
+      tmem_st16(tmem + lanes + ACOL + static_cast<uint32_t>(d * 16), a);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aready[d]);
+      ++j;
+      if (++s == NST) {
+        s = 0;
+        ph ^= 1u;
+      }
+      if (++d == NSLOT) {
+        d = 0;
+        dph ^= 1u;
+      }
+      more = walk_next(w, p, first, ntl);
+    }
+  } else {
+    // ------------------------------------------------------------ read back
+    // Warps 11..18, two per quarter of tensor-memory lanes: each reads half of
+    // a block's accumulator columns (rows of x), takes the block's scale
+    // from the stage (held until these warps let it go) and adds s * D.
+    const int q = warp & 3;
+    const int h = (warp - RB0) >> 2;  // which HR accumulator columns
+    const int c = 32 * q + lane;
+    const uint32_t lanes = static_cast<uint32_t>(32 * q) << 16;
+    // accumulators in pairs: the packed f32x2 FMA leaves the issue slots of
+    // this warp's scheduler to the MMA issuer (scalar FFMAs there starve
+    // tcgen05.mma issue), and takes half the instructions
+    float2 acc[HR / 2];
+#pragma unroll
+    for (int i = 0; i < HR / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+    bool waited = false;
+    Walk w{0, 0, 0, 0, 0, 0};
+    bool more = ntl > 0;
+    if (more) walk_load(w, p, first);
+    int s = 0, d = 0;
+    uint32_t ph = 0, dph = 0;
+#pragma unroll 1
+    while (more) {
+      bool okw = mbar_wait_bounded(&dready[d], dph, p.timeout_ns, abort_flag, p.err, K_TILE, 6);
+      if (okw) okw = mbar_wait_bounded(&full[s], ph, p.timeout_ns, abort_flag, p.err, K_TILE, 8);
+      if (!__all_sync(0xffffffffu, okw)) break;
+      tc_fence_after();
+      const float sc = *reinterpret_cast<const float*>(smem + s * SB + PB + 2048 + 4 * c);
+      const float2 sc2 = make_float2(sc, sc);
+      constexpr int CH = HR < 32 ? HR : 32;  // columns per tensor-memory load
+#pragma unroll
+      for (int k0 = 0; k0 < HR; k0 += CH) {
+        uint32_t v[CH];
+        tmem_ld_cols<CH>(tmem + lanes + static_cast<uint32_t>(d * NX + h * HR + k0), v);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (k0 + CH == HR) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&dfree[d]);
+            mbar_arrive(&empty[s]);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < CH / 2; ++i)
+          acc[k0 / 2 + i] = __ffma2_rn(sc2, make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
+                                       acc[k0 / 2 + i]);
+      }
+      if (++s == NST) {
+        s = 0;
+        ph ^= 1u;
+      }
+      if (++d == NSLOT) {
+        d = 0;
+        dph ^= 1u;
+      }
+      if (w.b == w.nb - 1) {
+        if (!waited) {
+          pdl_wait();  // y, bias and the residual follow the previous launch
+          waited = true;
+        }
+        const TMat& m = p.m[w.g];
+        const int64_t n = static_cast<int64_t>(w.ct) * TN + c;
+        const int r0 = w.xt * NX + h * HR;
+        if (n < m.N) {
+          const Epi e{m.bias, m.res, m.ldr, m.act, 0};
+          const int rows = m.M - r0;  // rows of this warp's half that exist
+          float* yp = m.y + static_cast<int64_t>(r0) * m.ldy + n;
+          if (epi_active(e)) {
+#pragma unroll
+            for (int i = 0; i < HR; ++i) {
+              const float v = (i & 1) ? acc[i / 2].y : acc[i / 2].x;
+              if (i < rows) *yp = epi_apply(v, e, r0 + i, n);
+              yp += m.ldy;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < HR; ++i) {
+              const float v = (i & 1) ? acc[i / 2].y : acc[i / 2].x;
+              if (i < rows) *yp = v;
+              yp += m.ldy;
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < HR / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+      }
+      more = walk_next(w, p, first, ntl);
+    }
+  }
+
+  // ---- teardown: copies landed, MMAs done, tensor-memory accesses complete
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS) : "memory");
+}
+
+// ---------------------------------------------------------------- x pieces
+
+struct SplitSrc {
+  const float* x;
+  uint8_t* dst;
+  int64_t ldx;
+  int64_t item0;  // first item of this source in the launch's numbering
+  int32_t M, K, nx, pad;
+};
+
+struct SplitParams {
+  SplitSrc s[TCAP];
+  int32_t count;
+  int64_t items;
+};
+
+// Top 8 significant bits of v as bf16 (v with its low 16 bits cleared).
+__device__ __forceinline__ uint32_t hi16(float v) { return __float_as_uint(v) & 0xFFFF0000u; }
+
+// One item: 8 consecutive k of one row of a row tile (zeros past M) -> three
+// 16-byte runs, one per piece, at their place in the operand layout.
+__global__ void __launch_bounds__(256) w4t_split_kernel(const __grid_constant__ SplitParams p) {
+  pdl_launch_dependents();
+  pdl_wait();  // x may be the previous launch's output
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < p.items;
+       it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int g = 0;
+    while (g + 1 < p.count && p.s[g + 1].item0 <= it) ++g;
+    const SplitSrc& S = p.s[g];
+    int64_t l = it - S.item0;
+    const int r = static_cast<int>(l & 7);
+    const int ks = static_cast<int>((l >> 3) & 1);
+    l >>= 4;
+    const int groups = S.nx >> 3;
+    const int gi = static_cast<int>(l % groups);
+    l /= groups;
+    const int hh = static_cast<int>(l & 1);
+    l >>= 1;
+    const int nb = S.K >> 5;
+    const int b = static_cast<int>(l % nb);
+    const int64_t xt = l / nb;
+    const int64_t row = xt * S.nx + 8 * gi + r;
+    const int k0 = 32 * b + 16 * hh + 8 * ks;
+    float v[8];
+    if (row < S.M) {
+      const float* src = S.x + row * S.ldx + k0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __ldg(src + e);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.f;
+    }
+    uint32_t w0[4], w1[4], w2[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t q0[2], q1[2], q2[2];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float x = v[2 * e + t];
+        q0[t] = hi16(x);
+        const float r1 = x - __uint_as_float(q0[t]);  // exact
+        q1[t] = hi16(r1);
+        q2[t] = __float_as_uint(r1 - __uint_as_float(q1[t]));  // exact, at most 8 significant bits
+      }
+      w0[e] = (q0[0] >> 16) | q0[1];
+      w1[e] = (q1[0] >> 16) | q1[1];
+      w2[e] = (q2[0] >> 16) | (q2[1] & 0xFFFF0000u);
+    }
+    uint8_t* d = S.dst + (xt * nb + b) * piece_bytes(S.nx) + hh * 32 * S.nx + gi * 256 + ks * 128 + r * 16;
+    *reinterpret_cast<uint4*>(d) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+    *reinterpret_cast<uint4*>(d + 64 * S.nx) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    *reinterpret_cast<uint4*>(d + 128 * S.nx) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- tile layout
+
+namespace {
+
+struct TileGeom {
+  int32_t nb, ntiles;
+  int64_t words;  // 32-bit words of the repacked buffer
+};
+
+bool tile_geom(int64_t K, int64_t N, TileGeom* g) {
+  if (K < 32 || K % 32 != 0 || K > (int64_t(1) << 24) || N <= 0 || N % 8 != 0 || N > (int64_t(1) << 23)) return false;
+  g->nb = static_cast<int32_t>(K / 32);
+  g->ntiles = static_cast<int32_t>((N + TN - 1) / TN);
+  g->words = static_cast<int64_t>(g->ntiles) * g->nb * (BLK / 4);
+  return true;
+}
+
+__device__ __constant__ int kNibPos[8] = {0, 16, 4, 20, 8, 24, 12, 28};
+
+__global__ void w4t_repack_kernel(const uint8_t* __restrict__ qw, const uint32_t* __restrict__ sc,
+                                  const uint32_t* __restrict__ zp, int64_t N, TileGeom g, uint32_t* __restrict__ out) {
+  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < g.words;
+       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t bid = o / (BLK / 4);  // tile * nb + block
+    const int w = static_cast<int>(o - bid * (BLK / 4));
+    const int64_t T = bid / g.nb;
+    const int64_t b = bid - T * g.nb;
+    uint32_t v = 0;
+    if (w < 512) {
+      const int64_t col = T * TN + (w >> 2);
+      const int j = w & 3;
+      if (col < N) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int64_t i = (b * 32 + 8 * j + r) * N + col;  // flat index of the nibble
+          const uint32_t q = (qw[i >> 1] >> ((i & 1) * 4)) & 0xFu;
+          v |= q << kNibPos[r];
+        }
+      }
+    } else if (w < 640) {
+      const int64_t col = T * TN + (w - 512);
+      if (col < N) v = sc[b * N + col];
+    } else {
+      const int64_t col = T * TN + 8 * (w - 640);
+      if (col < N) v = zp[(b * N + col) >> 3];
+    }
+    out[o] = v;
+  }
+}
+
+// page word pw of qw (8 nibbles: row k, columns c0 .. c0 + 7) from the tile layout
+__global__ void w4t_restore_qw_kernel(const uint32_t* __restrict__ in, int64_t K, int64_t N, TileGeom g,
+                                      uint32_t* __restrict__ qw) {
+  const int64_t words = K * N / 8;
+  for (int64_t pw = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; pw < words;
+       pw += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t k = (pw * 8) / N;
+    const int64_t c0 = pw * 8 - k * N;
+    const int64_t b = k >> 5;
+    const int j = static_cast<int>((k & 31) >> 3), r = static_cast<int>(k & 7);
+    uint32_t v = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t col = c0 + i;
+      const int64_t T = col / TN;
+      const uint32_t word = in[(T * g.nb + b) * (BLK / 4) + (col - T * TN) * 4 + j];
+      v |= ((word >> kNibPos[r]) & 0xFu) << (4 * i);
+    }
+    qw[pw] = v;
+  }
+}
+
+__global__ void w4t_restore_sz_kernel(const uint32_t* __restrict__ in, int64_t N, TileGeom g, uint32_t* __restrict__ sc,
+                                      uint32_t* __restrict__ zp) {
+  const int64_t n_sc = static_cast<int64_t>(g.nb) * N;
+  const int64_t n_zp = n_sc / 8;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n_sc + n_zp;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (e < n_sc) {
+      const int64_t b = e / N, col = e - b * N, T = col / TN;
+      sc[e] = in[(T * g.nb + b) * (BLK / 4) + 512 + (col - T * TN)];
+    } else {
+      const int64_t z = e - n_sc;
+      const int64_t b = (z * 8) / N, col = z * 8 - b * N, T = col / TN;
+      zp[z] = in[(T * g.nb + b) * (BLK / 4) + 640 + (col - T * TN) / 8];
+    }
+  }
+}
+
+bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// ---------------------------------------------------------------- host plan
+
+// Rows of x per row tile: the smallest MMA N of 16, 32, 64, 128 that holds M
+// (row tiles of 128 beyond).
+int rows_per_tile(int64_t M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+
+int64_t pieces_bytes(int64_t M, int64_t K) {
+  const int nx = rows_per_tile(M);
+  return (M + nx - 1) / nx * nx * K * 6;
+}
+
+constexpr int64_t kPieceAlign = 256;
+constexpr int64_t kMaxRowTiles = 1024;
+
+int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+bool active(const w4r_desc& d) { return d.M > 0 && d.N > 0 && d.K > 0; }
+
+bool same_x(const w4r_desc& a, const w4r_desc& b) {
+  return a.x == b.x && a.ldx == b.ldx && a.M == b.M && a.K == b.K;
+}
+
+// Workspace offset of each descriptor's pieces (-1: none); one set of pieces
+// per distinct (x, ldx, M, K). Returns the bytes needed.
+int64_t assign_pieces(const w4r_desc* d, int count, std::vector<int64_t>* off) {
+  off->assign(count, -1);
+  int64_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    if (!active(d[i])) continue;
+    for (int k = 0; k < i; ++k)
+      if ((*off)[k] >= 0 && same_x(d[k], d[i])) {
+        (*off)[i] = (*off)[k];
+        break;
+      }
+    if ((*off)[i] >= 0) continue;
+    (*off)[i] = total;
+    total += round_up(pieces_bytes(d[i].M, d[i].K), kPieceAlign);
+  }
+  return total;
+}
+
+// The tiles of a launch over G CTAs: every tile goes to the CTA with the
+// fewest blocks so far, largest tiles first (ties to the lower tile number,
+// then the lower CTA), and each CTA takes its tiles in tile order.
+void plan_tiles(const std::vector<uint32_t>& tiles, const std::vector<int>& cost, int G, TParams* prm) {
+  const int T = static_cast<int>(tiles.size());
+  std::vector<int> order(T);
+  for (int t = 0; t < T; ++t) order[t] = t;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  using Slot = std::pair<int64_t, int>;
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+  for (int c = 0; c < G; ++c) heap.push({0, c});
+  std::vector<std::vector<int>> per(G);
+  for (int t : order) {
+    Slot sl = heap.top();
+    heap.pop();
+    per[sl.second].push_back(t);
+    sl.first += cost[t];
+    heap.push(sl);
+  }
+  uint32_t pos = 0;
+  for (int c = 0; c < G; ++c) {
+    std::sort(per[c].begin(), per[c].end());
+    prm->first[c] = pos;
+    for (int t : per[c]) prm->list[pos++] = tiles[t];
+  }
+  prm->first[G] = pos;
+}
+
+struct Launch {
+  int nx = 0;
+  int grid = 0;
+  TParams prm;
+};
+
+// The launches of one call: x pieces first (one split launch per TCAP
+// sources), then the tile GEMMs, one per rows-per-tile class and run of at
+// most TCAP matrices and LCAP tiles.
+struct CallPlan {
+  int dev = -1;
+  uint64_t used = 0;
+  std::vector<w4r_desc> descs;
+  const void* ws = nullptr;
+  std::vector<SplitParams> splits;
+  std::vector<std::unique_ptr<Launch>> gemms;
+};
+
+bool same_descs(const std::vector<w4r_desc>& a, const w4r_desc* b, int count) {
+  if (static_cast<int>(a.size()) != count) return false;
+  for (int i = 0; i < count; ++i) {
+    const w4r_desc& p = a[i];
+    const w4r_desc& q = b[i];
+    if (p.x != q.x || p.ldx != q.ldx || p.wr != q.wr || p.y != q.y || p.ldy != q.ldy || p.M != q.M || p.K != q.K ||
+        p.N != q.N || p.bias != q.bias || p.residual != q.residual || p.ldr != q.ldr || p.act != q.act)
+      return false;
+  }
+  return true;
+}
+
+void build_plan(const w4r_desc* d, int count, void* ws, int sms, w4dev::ErrorWord* err, CallPlan* cp) {
+  cp->splits.clear();
+  cp->gemms.clear();
+  std::vector<int64_t> off;
+  assign_pieces(d, count, &off);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  // split launches: distinct sources
+  SplitParams sp;
+  std::memset(&sp, 0, sizeof(sp));
+  for (int i = 0; i < count; ++i) {
+    if (!active(d[i])) continue;
+    bool dup = false;
+    for (int k = 0; k < i; ++k)
+      if (active(d[k]) && off[k] == off[i]) dup = true;
+    if (dup) continue;
+    if (sp.count == TCAP) {
+      cp->splits.push_back(sp);
+      std::memset(&sp, 0, sizeof(sp));
+    }
+    SplitSrc& s = sp.s[sp.count++];
+    const int nx = rows_per_tile(d[i].M);
+    s.x = d[i].x;
+    s.dst = base + off[i];
+    s.ldx = d[i].ldx;
+    s.item0 = sp.items;
+    s.M = static_cast<int32_t>(d[i].M);
+    s.K = static_cast<int32_t>(d[i].K);
+    s.nx = nx;
+    sp.items += (d[i].M + nx - 1) / nx * nx * (d[i].K / 8);
+  }
+  if (sp.count > 0) cp->splits.push_back(sp);
+  // GEMM launches per rows-per-tile class
+  for (int nx : {16, 32, 64, 128}) {
+    std::vector<uint32_t> tiles;
+    std::vector<int> cost;
+    std::unique_ptr<Launch> L;
+    int nm = 0;
+    auto flush = [&]() {
+      if (L && !tiles.empty()) {
+        const int T = static_cast<int>(tiles.size());
+        L->grid = std::min(std::min(sms, 256), T);
+        plan_tiles(tiles, cost, L->grid, &L->prm);
+        L->prm.err = err;
+        cp->gemms.push_back(std::move(L));
+      }
+      L.reset(new Launch);
+      std::memset(&L->prm, 0, sizeof(L->prm));
+      L->nx = nx;
+      tiles.clear();
+      cost.clear();
+      nm = 0;
+    };
+    flush();
+    for (int i = 0; i < count; ++i) {
+      if (!active(d[i]) || rows_per_tile(d[i].M) != nx) continue;
+      TileGeom g;
+      tile_geom(d[i].K, d[i].N, &g);
+      const int64_t nxt = (d[i].M + nx - 1) / nx;
+      // a matrix with more tiles than one launch holds is cut by row tiles
+      int64_t xt0 = 0;
+      while (xt0 < nxt) {
+        const int64_t room = (LCAP - static_cast<int64_t>(tiles.size())) / g.ntiles;
+        if (room == 0 || nm == TCAP) {
+          flush();
+          continue;
+        }
+        const int64_t xt1 = std::min(nxt, xt0 + room);
+        TMat& m = L->prm.m[nm];
+        m.wt = static_cast<const uint8_t*>(d[i].wr);
+        m.xp = base + off[i];
+        m.y = d[i].y;
+        m.bias = d[i].bias;
+        m.res = d[i].residual;
+        m.ldy = d[i].ldy;
+        m.ldr = d[i].ldr;
+        m.M = static_cast<int32_t>(d[i].M);
+        m.N = static_cast<int32_t>(d[i].N);
+        m.nb = g.nb;
+        m.act = d[i].act;
+        for (int64_t xt = xt0; xt < xt1; ++xt)
+          for (int ct = 0; ct < g.ntiles; ++ct) {
+            tiles.push_back((static_cast<uint32_t>(nm) << 26) | (static_cast<uint32_t>(xt) << 16) |
+                            static_cast<uint32_t>(ct));
+            cost.push_back(g.nb);
+          }
+        ++nm;
+        xt0 = xt1;
+      }
+    }
+    flush();
+  }
+}
+
+template <int NX>
+w4_status launch_gemm_nx(const Launch& L, cudaStream_t st, const w4host::DeviceInfo& di) {
+  using namespace w4host;
+  static int configured[64] = {};
+  if (di.dev < 64 && !configured[di.dev]) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(w4t_gemm_kernel<NX>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(w4t_gemm)");
+    configured[di.dev] = 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(L.grid));
+  cfg.blockDim = dim3(block_threads(NX));
+  cfg.dynamicSmemBytes = static_cast<size_t>(SMEM_BYTES);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, w4t_gemm_kernel<NX>, L.prm);
+  return e == cudaSuccess ? W4_OK : cuda_fail(e, "launch w4t_gemm");
+}
+
+w4_status launch_split(const SplitParams& sp, cudaStream_t st, const w4host::DeviceInfo& di) {
+  using namespace w4host;
+  const int64_t blocks = std::min<int64_t>((sp.items + 255) / 256, static_cast<int64_t>(di.sms) * 16);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(blocks, 1)));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, w4t_split_kernel, sp);
+  return e == cudaSuccess ? W4_OK : cuda_fail(e, "launch w4t_split");
+}
+
+w4_status check_tdesc(const w4r_desc& d) {
+  using namespace w4host;
+  if (d.M < 0 || d.K < 0 || d.N < 0) return fail(W4_ERR_SHAPE, "negative size");
+  if (d.act < W4_ACT_NONE || d.act > W4_ACT_GELU_ERF) return fail(W4_ERR_VALUE, "unknown activation %d", int(d.act));
+  if (d.reserved != 0) return fail(W4_ERR_VALUE, "reserved field must be 0");
+  if (d.M == 0 || d.N == 0) return W4_OK;
+  if (d.K == 0) {
+    if (d.y == nullptr) return fail(W4_ERR_NULL, "y must not be NULL");
+  } else {
+    TileGeom g;
+    if (!tile_geom(d.K, d.N, &g))
+      return fail(W4_ERR_SHAPE, "the tile layout takes K %% 32 == 0, N %% 8 == 0, K <= 2^24, N <= 2^23 (K=%lld N=%lld)",
+                  (long long)d.K, (long long)d.N);
+    if (d.x == nullptr || d.wr == nullptr || d.y == nullptr) return fail(W4_ERR_NULL, "x, wr and y must not be NULL");
+    if (d.ldx < d.K) return fail(W4_ERR_SHAPE, "ldx < K");
+    if ((d.M + rows_per_tile(d.M) - 1) / rows_per_tile(d.M) > kMaxRowTiles)
+      return fail(W4_ERR_SHAPE, "M above %lld rows", (long long)(kMaxRowTiles * 128));
+    if (!aligned_to(d.x, 4)) return fail(W4_ERR_ALIGN, "x must be 4-byte aligned");
+    if (!aligned_to(d.wr, 16)) return fail(W4_ERR_ALIGN, "the tile-layout weight must be 16-byte aligned");
+  }
+  if (d.ldy < d.N) return fail(W4_ERR_SHAPE, "ldy < N");
+  if (!aligned_to(d.y, 4)) return fail(W4_ERR_ALIGN, "y must be 4-byte aligned");
+  if ((d.bias != nullptr && !aligned_to(d.bias, 4)) || (d.residual != nullptr && !aligned_to(d.residual, 4)))
+    return fail(W4_ERR_ALIGN, "bias and residual must be 4-byte aligned");
+  if (d.residual != nullptr && d.ldr < d.N) return fail(W4_ERR_SHAPE, "ldr < N");
+  return W4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t w4t_repacked_bytes(int64_t K, int64_t N) {
+  TileGeom g;
+  return tile_geom(K, N, &g) ? static_cast<size_t>(g.words) * 4 : 0;
+}
+
+w4_status w4t_repack(const uint8_t* qw, const float* scales, const uint8_t* zp, int64_t K, int64_t N, void* wt,
+                     void* stream) {
+  using namespace w4host;
+  TileGeom g;
+  if (!tile_geom(K, N, &g)) return fail(W4_ERR_SHAPE, "the tile layout takes K %% 32 == 0, N %% 8 == 0");
+  if (qw == nullptr || scales == nullptr || zp == nullptr || wt == nullptr) return fail(W4_ERR_NULL, "NULL buffer");
+  if (!aligned_to(qw, 16) || !aligned_to(scales, 16) || !aligned_to(zp, 16) || !aligned_to(wt, 16))
+    return fail(W4_ERR_ALIGN, "qw, scales, zp and wt must be 16-byte aligned");
+  const DeviceInfo* di = nullptr;
+  w4_status rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  const int64_t blocks = std::min<int64_t>((g.words + 255) / 256, static_cast<int64_t>(di->sms) * 32);
+  w4t_repack_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      qw, reinterpret_cast<const uint32_t*>(scales), reinterpret_cast<const uint32_t*>(zp), N, g,
+      static_cast<uint32_t*>(wt));
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W4_OK : cuda_fail(e, "launch w4t_repack");
+}
+
+w4_status w4t_repack_restore(const void* wt, int64_t K, int64_t N, uint8_t* qw, float* scales, uint8_t* zp,
+                             void* stream) {
+  using namespace w4host;
+  TileGeom g;
+  if (!tile_geom(K, N, &g)) return fail(W4_ERR_SHAPE, "the tile layout takes K %% 32 == 0, N %% 8 == 0");
+  if (qw == nullptr || scales == nullptr || zp == nullptr || wt == nullptr) return fail(W4_ERR_NULL, "NULL buffer");
+  if (!aligned_to(qw, 16) || !aligned_to(scales, 16) || !aligned_to(zp, 16) || !aligned_to(wt, 16))
+    return fail(W4_ERR_ALIGN, "qw, scales, zp and wt must be 16-byte aligned");
+  const DeviceInfo* di = nullptr;
+  w4_status rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t cap = static_cast<int64_t>(di->sms) * 32;
+  const int64_t qwords = K * N / 8;
+  w4t_restore_qw_kernel<<<static_cast<unsigned>(std::min<int64_t>((qwords + 255) / 256, cap)), 256, 0, st>>>(
+      static_cast<const uint32_t*>(wt), K, N, g, reinterpret_cast<uint32_t*>(qw));
+  const int64_t sz = static_cast<int64_t>(g.nb) * N + static_cast<int64_t>(g.nb) * N / 8;
+  w4t_restore_sz_kernel<<<static_cast<unsigned>(std::min<int64_t>((sz + 255) / 256, cap)), 256, 0, st>>>(
+      static_cast<const uint32_t*>(wt), N, g, reinterpret_cast<uint32_t*>(scales), reinterpret_cast<uint32_t*>(zp));
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W4_OK : cuda_fail(e, "launch w4t_restore");
+}
+
+size_t w4t_workspace_size(const w4t_desc* descs, int32_t count) {
+  if (descs == nullptr || count <= 0) return 0;
+  std::vector<int64_t> off;
+  return static_cast<size_t>(assign_pieces(descs, count, &off));
+}
+
+w4_status w4t_matmul_grouped(const w4t_desc* descs, int32_t count, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  using namespace w4host;
+  if (count < 0) return fail(W4_ERR_SHAPE, "negative count");
+  if (count == 0) return W4_OK;
+  if (descs == nullptr) return fail(W4_ERR_NULL, "descs is NULL");
+  int work = 0, zero_k = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    const w4_status rc = check_tdesc(descs[i]);
+    if (rc != W4_OK) {
+      char why[256];
+      snprintf(why, sizeof(why), "%s", w4_last_error());
+      return fail(rc, "descriptor %d: %s", i, why);
+    }
+    if (active(descs[i])) ++work;
+    if (descs[i].M > 0 && descs[i].N > 0 && descs[i].K == 0) ++zero_k;
+  }
+  if (work == 0 && zero_k == 0) return W4_OK;
+  std::vector<int64_t> off;
+  const int64_t need = assign_pieces(descs, count, &off);
+  if (need > 0) {
+    if (workspace == nullptr) return fail(W4_ERR_WORKSPACE, "workspace is NULL, %lld bytes needed", (long long)need);
+    if (!aligned_to(workspace, 16)) return fail(W4_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+    if (static_cast<int64_t>(workspace_bytes) < need)
+      return fail(W4_ERR_WORKSPACE, "workspace of %zu bytes, %lld needed", workspace_bytes, (long long)need);
+  }
+  const DeviceInfo* di = nullptr;
+  w4_status rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int32_t i = 0; i < count; ++i) {
+    const w4r_desc& d = descs[i];
+    if (d.M > 0 && d.N > 0 && d.K == 0) {
+      w4_desc z{};
+      z.y = d.y;
+      z.ldy = d.ldy;
+      z.M = d.M;
+      z.N = d.N;
+      z.bias = d.bias;
+      z.residual = d.residual;
+      z.ldr = d.ldr;
+      z.act = d.act;
+      rc = launch_zero_fill(d.y, d.ldy, d.M, d.N, st, &z);
+      if (rc != W4_OK) return rc;
+    }
+  }
+  if (work == 0) return W4_OK;
+
+  static thread_local std::unique_ptr<CallPlan[]> cache;
+  static thread_local uint64_t clock = 0;
+  constexpr int kEntries = 4;
+  if (!cache) cache.reset(new CallPlan[kEntries]);
+  ++clock;
+  CallPlan* hit = nullptr;
+  for (int e = 0; e < kEntries && hit == nullptr; ++e)
+    if (cache[e].dev == di->dev && cache[e].ws == workspace && same_descs(cache[e].descs, descs, count)) hit = &cache[e];
+  if (hit == nullptr) {
+    int victim = 0;
+    for (int e = 1; e < kEntries; ++e)
+      if (cache[e].used < cache[victim].used) victim = e;
+    CallPlan& cp = cache[victim];
+    cp.dev = -1;
+    build_plan(descs, count, workspace, di->sms, di->err, &cp);
+    cp.descs.assign(descs, descs + count);
+    cp.ws = workspace;
+    cp.dev = di->dev;
+    hit = &cp;
+  }
+  hit->used = clock;
+  const uint64_t tmo = wait_timeout_ns();
+  for (const SplitParams& sp : hit->splits) {
+    rc = launch_split(sp, st, *di);
+    if (rc != W4_OK) return rc;
+  }
+  for (auto& L : hit->gemms) {
+    L->prm.timeout_ns = tmo;
+    switch (L->nx) {
+      case 16: rc = launch_gemm_nx<16>(*L, st, *di); break;
+      case 32: rc = launch_gemm_nx<32>(*L, st, *di); break;
+      case 64: rc = launch_gemm_nx<64>(*L, st, *di); break;
+      default: rc = launch_gemm_nx<128>(*L, st, *di); break;
+    }
+    if (rc != W4_OK) return rc;
+  }
+  return W4_OK;
+}
+
+w4_status w4t_matmul(const w4t_desc* d, void* workspace, size_t workspace_bytes, void* stream) {
+  return w4t_matmul_grouped(d, 1, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
