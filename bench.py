@@ -632,9 +632,22 @@ def config2(peaks, budget):
     return out
 
 
+def tile_roofline(tf: float, peaks: dict, kernel: str) -> dict:
+    """Roofline of the tile GEMM: algorithmic 2MKN flops against the tf32
+    peak, and the bf16 MMA flops it issues (three per product) against the
+    bf16 peak."""
+    pk = tf32_peak(peaks)
+    return {"kernel": kernel, "bound": "tensor", "achieved": round(tf, 2), "unit": "TFLOP/s",
+            "achieved_note": "algorithmic 2MKN flops", "peak": round(pk, 1),
+            "peak_note": "tf32 dense = bf16 peak x 1.1 / 2.25", "frac": round(tf / pk, 4),
+            "issued_bf16": round(3 * tf, 2), "peak_bf16": peaks["bf16_tflops"],
+            "frac_issued_bf16": round(3 * tf / peaks["bf16_tflops"], 4)}
+
+
 def config3(peaks, budget, wl):
-    """GPT-2 prefill: M = 58 rows through the 48 weights (tensor cores, grouped),
-    then the head on row 57 of the last layer's output (streaming head)."""
+    """GPT-2 prefill: M = 58 rows through the 48 weights (tile layout, tensor
+    cores, grouped), then the head on row 57 of the last layer's output
+    (streaming head)."""
     import torch
     import int8_weight_quantized_w4_b200 as w4
     import oracle
@@ -647,36 +660,36 @@ def config3(peaks, budget, wl):
     steps = []
     for r, cp in enumerate(wl.copies):
         ws = cp[3]
-        descs = w4.make_descs([{"x": xs[i], "y": ys[i], "K": K_, "N": N_, **ws[i]}
-                               for i, (_, K_, N_) in enumerate(wl.shapes)])
+        wts = [w4.w4t_repack(ws[i]["qw"], ws[i]["scales"], ws[i]["zp"], K_, N_)
+               for i, (_, K_, N_) in enumerate(wl.shapes)]
+        descs = w4.make_rdescs([{"x": xs[i], "y": ys[i], "wr": wts[i], "K": K_, "N": N_}
+                                for i, (_, K_, N_) in enumerate(wl.shapes)])
         tr = w4.i8_head_repack(cp[1], cp[2], K, V)
-        steps.append((descs, tr))
+        steps.append((descs, tr, wts))
+    scratch = torch.empty(max(w4.w4t_workspace_size(steps[0][0]), 16), dtype=torch.uint8, device=dev)
     h = ys[-1][M - 1:M]
     lg = torch.empty((1, V), device=dev)
 
-    def step(hs, d=None, tr=None):
-        _ok(lib.w4_matmul_grouped(d, len(d), None, 0, hs), lib, "w4_matmul_grouped")
+    def body(hs, d):
+        _ok(lib.w4t_matmul_grouped(d, len(d), scratch.data_ptr(), scratch.numel(), hs), lib, "w4t_matmul_grouped")
+
+    def step(hs, d, tr):
+        body(hs, d)
         _ok(lib.i8r_head_logits(h.data_ptr(), tr.data_ptr(), K, V, lg.data_ptr(), hs), lib, "i8r_head_logits")
 
-    def body_only(hs, d=None):
-        _ok(lib.w4_matmul_grouped(d, len(d), None, 0, hs), lib, "w4_matmul_grouped")
-
-    ms = graph_ms([lambda hs, d=d, tr=tr: step(hs, d, tr) for d, tr in steps], 20)
-    msb = graph_ms([lambda hs, d=d: body_only(hs, d) for d, _ in steps], 20)
+    ms = graph_ms([lambda hs, d=d, tr=tr: step(hs, d, tr) for d, tr, _ in steps], 20)
+    msb = graph_ms([lambda hs, d=d: body(hs, d) for d, _, _ in steps], 20)
     flops = 2.0 * M * sum(K_ * N_ for _, K_, N_ in wl.shapes)
     tf = flops / (msb * 1e-3) / 1e12
-    pk = tf32_peak(peaks)
     W = synth.w4_weight(3072, 768, 3)
     xh = synth.activations(M, 3072, 3)
     rate, n, el = _oracle_rate(lambda: oracle.w4_matmul_ref(xh, W["qw"], W["scales"], W["zp"], 3072, 768),
                                2.0 * M * 3072 * 768 / 1e12, budget)
-    return {"workload": "GPT-2 prefill: M=58 through the 48 W4 weights (tcgen05 3xTF32, grouped) + int8 head "
-                        "on row 57 of the last output (streaming head)",
+    return {"workload": "GPT-2 prefill: M=58 through the 48 W4 weights (tile layout, tcgen05 bf16 with an exact "
+                        "three-piece split of x, grouped) + int8 head on row 57 of the last output (streaming head)",
             "metric": "prefill TFLOP/s (algorithmic 2MKN, body)", "value": round(tf, 2), "unit": "TFLOP/s",
             "us_per_step": round(ms * 1e3, 2), "us_body": round(msb * 1e3, 2),
-            "roofline": {"kernel": "w4_tc_kernel (tcgen05.mma kind::tf32, 3 MMAs per product)", "bound": "tensor",
-                         "achieved": round(3 * tf, 2), "achieved_note": "tf32 MMA flops issued: 3x algorithmic",
-                         "peak": round(pk, 1), "unit": "TFLOP/s", "frac": round(3 * tf / pk, 4)},
+            "roofline": tile_roofline(tf, peaks, "w4t_gemm_kernel<64> (tcgen05.mma kind::f16, 3 MMAs per product)"),
             "cpu_baseline": _cpu(round(rate, 6), "TFLOP/s", "oracle w4_matmul_ref, one 3072x768 weight at M=58",
                                  n, el)}
 
@@ -684,7 +697,8 @@ def config3(peaks, budget, wl):
 def config4(peaks, budget, clocks):
     """3.8B-dense-shaped stack, 32 layers x [3072x9216, 3072x3072, 3072x16384,
     8192x3072]: decode at M = 1 (streaming layout), 8 (split-K GEMV) and 32
-    (tensor cores), prefill at M = 2048 (tensor cores). 128 distinct weights
+    (tile layout, tensor cores), prefill at M = 2048 (tile layout, tensor
+    cores). 128 distinct weights
     (2.32 GB: L2-cold by size), generated on the GPU with a seeded generator
     in the synthetic distributions (uniform nibbles, scales U[0.005, 0.02])."""
     import torch
@@ -719,8 +733,19 @@ def config4(peaks, budget, clocks):
                         "roofline": {"kernel": "w4r_gemv_m1_kernel", "bound": "hbm", "achieved": round(g1, 1),
                                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                      "frac": round(g1 / peaks["hbm_gbs"], 4)}}
-    # decode M = 8 (split-K GEMV) and M = 32 (tensor cores), page format
-    for M in (8, 32):
+    # the tile layout of the 128 weights, for M = 32 and the prefill
+    wts = [w4.w4t_repack(Wd["qw"], Wd["scales"], Wd["zp"], K, N) for Wd, (K, N) in zip(weights, shapes)]
+
+    def tile_ms(M, reps):
+        xm = {K: torch.randn((M, K), device=dev, generator=gen) for K in (3072, 8192)}
+        ym = [torch.empty((M, N), device=dev) for _, N in shapes]
+        td = w4.make_rdescs([{"x": xm[K], "wr": wts[i], "y": ym[i], "K": K, "N": N} for i, (K, N) in enumerate(shapes)])
+        scratch = torch.empty(max(w4.w4t_workspace_size(td), 16), dtype=torch.uint8, device=dev)
+        return graph_ms([lambda hs: _ok(lib.w4t_matmul_grouped(td, len(td), scratch.data_ptr(), scratch.numel(), hs),
+                                        lib, "w4t_matmul_grouped")], reps)
+
+    # decode M = 8 (split-K GEMV, page format)
+    for M in (8,):
         xm = {K: torch.randn((M, K), device=dev, generator=gen) for K in (3072, 8192)}
         ym = [torch.empty((M, N), device=dev) for _, N in shapes]
         items = [{"x": xm[K], "y": ym[i], "K": K, "N": N, **weights[i]} for i, (K, N) in enumerate(shapes)]
@@ -731,35 +756,29 @@ def config4(peaks, budget, clocks):
                                        "w4_matmul_grouped")], 5)
         tfl = 2.0 * M * wsum / (msm * 1e-3) / 1e12
         gb = nbytes / (msm * 1e-3) / 1e9
-        if M == 8:
-            pk = fp32_alu_peak_tflops(clocks.get("sm_mhz"))
-            roof = {"kernel": "w4_gemv_kernel<8> (split-K GEMV)", "bound": "alu", "achieved": round(tfl, 2),
-                    "peak": round(pk, 1), "unit": "TFLOP/s", "frac": round(tfl / pk, 4),
-                    "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x the sampled SM clock"}
-        else:
-            pk = tf32_peak(peaks)
-            roof = {"kernel": "w4_tc_kernel (3xTF32)", "bound": "tensor", "achieved": round(3 * tfl, 2),
-                    "achieved_note": "tf32 MMA flops issued: 3x algorithmic", "peak": round(pk, 1),
-                    "unit": "TFLOP/s", "frac": round(3 * tfl / pk, 4)}
+        pk = fp32_alu_peak_tflops(clocks.get("sm_mhz"))
+        roof = {"kernel": "w4_gemv_kernel<8> (split-K GEMV)", "bound": "alu", "achieved": round(tfl, 2),
+                "peak": round(pk, 1), "unit": "TFLOP/s", "frac": round(tfl / pk, 4),
+                "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x the sampled SM clock"}
         out[f"decode_M{M}"] = {"metric": "TFLOP/s (algorithmic 2MKN)", "value": round(tfl, 2), "unit": "TFLOP/s",
                                "weight_GB_per_s": round(gb, 1), "ms_per_step": round(msm, 4), "roofline": roof}
         del xm, ym, items, descs, ws
-    # prefill M = 2048 (tensor cores): x shared by the weights of one K, y distinct per weight
+    # decode M = 32 on the tile layout (tensor cores, 32-row tiles)
+    M = 32
+    msm = tile_ms(M, 5)
+    tfl = 2.0 * M * wsum / (msm * 1e-3) / 1e12
+    out["decode_M32"] = {"metric": "TFLOP/s (algorithmic 2MKN)", "value": round(tfl, 2), "unit": "TFLOP/s",
+                         "weight_GB_per_s": round(nbytes / (msm * 1e-3) / 1e9, 1), "ms_per_step": round(msm, 4),
+                         "roofline": tile_roofline(tfl, peaks, "w4t_gemm_kernel<32> (tcgen05.mma kind::f16)")}
+    # prefill M = 2048 on the tile layout: x shared by the weights of one K
+    # (its pieces made once per call), y distinct per weight
     M = 2048
-    xp = {K: torch.randn((M, K), device=dev, generator=gen) for K in (3072, 8192)}
-    yp = [torch.empty((M, N), device=dev) for _, N in shapes]
-    descs = w4.make_descs([{"x": xp[K], "y": yp[i], "K": K, "N": N, **weights[i]} for i, (K, N) in enumerate(shapes)])
-    msp = graph_ms([lambda hs: _ok(lib.w4_matmul_grouped(descs, len(descs), None, 0, hs), lib, "w4_matmul_grouped")], 2)
+    msp = tile_ms(M, 2)
     tfp = 2.0 * M * wsum / (msp * 1e-3) / 1e12
-    pk = tf32_peak(peaks)
     out["prefill_M2048"] = {"metric": "prefill TFLOP/s (algorithmic 2MKN)", "value": round(tfp, 2), "unit": "TFLOP/s",
                             "ms_per_step": round(msp, 3),
-                            "roofline": {"kernel": "w4_tc_kernel (tcgen05.mma kind::tf32, 3 MMAs per product)",
-                                         "bound": "tensor", "achieved": round(3 * tfp, 1),
-                                         "achieved_note": "tf32 MMA flops issued: 3x algorithmic",
-                                         "peak": round(pk, 1), "unit": "TFLOP/s", "frac": round(3 * tfp / pk, 4),
-                                         "frac_algorithmic": round(tfp / pk, 4)}}
-    del xp, yp, descs, weights
+                            "roofline": tile_roofline(tfp, peaks, "w4t_gemm_kernel<128> (tcgen05.mma kind::f16)")}
+    del wts, weights
     torch.cuda.empty_cache()
     # the oracle on one o_proj weight (3072x3072) at each M, scaled to the metric
     W = synth.w4_weight(3072, 3072, 38)
@@ -908,98 +927,6 @@ def run_reference(args, world, rank):
             "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-# ---------------------------------------------------------------- prefill
-
-PREFILL_M = 2048
-PREFILL_LAYERS = 32
-PREFILL_SHAPES = [(3072, 9216), (3072, 3072), (3072, 16384), (8192, 3072)]  # qkv, o, gate_up, down
-
-
-def run_prefill(args):
-    """The 3.8B-dense-shaped W4 stack as prefill: 32 layers x 4 weights at
-    M = 2048 through the tensor-core (tcgen05, 3xTF32) path, one grouped call
-    per 48 weights. The 4 weight shapes of a layer are generated once (seeded)
-    and serve all 32 layers; x and y are shared by weights of the same K or N.
-    Metric: algorithmic TFLOP/s (2 M K N), against the tf32 tensor roofline."""
-    import torch
-
-    import int8_weight_quantized_w4_b200 as w4
-    from int8_weight_quantized_w4_b200 import synth
-    M = PREFILL_M
-    dev = torch.device("cuda", 0)
-    weights = []
-    for i, (K, N) in enumerate(PREFILL_SHAPES):
-        W = synth.w4_weight(K, N, 3800 + i)
-        weights.append({k: torch.from_numpy(W[k]).to(dev) for k in ("qw", "scales", "zp")})
-    xs = {K: torch.from_numpy(synth.activations(M, K, 3900 + K)).to(dev) for K, _ in PREFILL_SHAPES}
-    ys = {N: torch.empty((M, N), dtype=torch.float32, device=dev) for _, N in PREFILL_SHAPES}
-    items = []
-    for _ in range(PREFILL_LAYERS):
-        for (K, N), Wd in zip(PREFILL_SHAPES, weights):
-            items.append(dict(x=xs[K], y=ys[N], K=K, N=N, **Wd))
-    descs = w4.make_descs(items)
-    lib = w4.lib()
-    st = torch.cuda.current_stream()
-
-    def step():
-        r = lib.w4_matmul_grouped(descs, len(items), None, 0, int(st.cuda_stream))
-        if r != 0:
-            raise RuntimeError(f"w4_matmul_grouped failed: {r} {lib.w4_last_error()}")
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize()
-    sampler = ClockSampler(gpu_id(0))
-    sampler.start()
-    time.sleep(0.2)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(st)
-    for _ in range(args.steps):
-        step()
-    t1.record(st)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    ms = t0.elapsed_time(t1) / args.steps
-    flops = 2.0 * M * PREFILL_LAYERS * sum(K * N for K, N in PREFILL_SHAPES)
-    tflops = flops / (ms * 1e-3) / 1e12
-    peaks = measured_peaks()
-    # the burst figure: this kernel keeps the tensor pipe well below the
-    # power cap, and its SM clock stays at the maximum (see "clocks")
-    tf32_peak = peaks["bf16_tflops"] * (1.1 / 2.25)  # nominal dense tf32 : bf16 ratio of the part
-    return {
-        "metric": "prefill TFLOP/s (3.8B-dense-shaped W4 stack, M=2048, fp32 via 3xTF32)",
-        "value": round(tflops, 2),
-        "unit": "TFLOP/s",
-        "n_gpus": 1,
-        "steps": args.steps,
-        "warmup": max(3, args.warmup),
-        "ms_per_step": round(ms, 4),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "f32 (3xTF32 tensor-core products, fp32 accumulation)",
-        "data": "synthetic (seeded uniform nibbles, fp32 N(0,1) activations)",
-        "config": {
-            "workload": "3.8B-dense-shaped W4 stack prefill: 32 layers x [3072x9216, 3072x3072, 3072x16384, "
-                        "8192x3072] at M=2048, grouped calls of 48 weights",
-            "weights": "the 4 shapes of one layer generated once, used by all 32 layers",
-            "algorithmic_tflop_per_step": round(flops / 1e12, 3),
-        },
-        "roofline": {
-            "kernel": "w4_tc_kernel (tcgen05.mma kind::tf32, 3 MMAs per product)",
-            "bound": "tensor",
-            "achieved": round(3 * tflops, 1),
-            "achieved_note": "tf32 MMA flops issued: 3x the algorithmic 2MKN",
-            "peak": round(tf32_peak, 1),
-            "peak_source": f"{peaks['_source']} bf16 cuBLAS (burst) x 1.1/2.25 nominal tf32:bf16",
-            "unit": "TFLOP/s",
-            "frac": round(3 * tflops / tf32_peak, 4),
-        },
-        "clocks": clocks,
-    }
-
-
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1011,12 +938,7 @@ def main():
                     help="device seconds of the timed step replays (the body and head alone get half each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config measurements (configs 0, 2, 3, 4)")
-    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
-                    help="decode: the GPT-2 decode step (the headline); prefill: the 3.8B-shaped stack at M=2048")
     args = ap.parse_args()
-    if args.workload == "prefill":
-        print(json.dumps(run_prefill(args)), flush=True)
-        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
