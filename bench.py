@@ -927,6 +927,52 @@ def run_reference(args, world, rank):
             "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def profile_case(name: str, calls: int) -> None:
+    """Run one workload's kernels `calls` times (no timing, no output but one
+    line) so that a profiler can capture them: "body" (the 48 GPT-2 weights
+    in the streaming layout, M = 1), "head" (the int8 head, streaming
+    layout, M = 1), "prefill-gpt2" (the 48 weights in the tile layout at
+    M = 58), "prefill-3p8b" (one 3.8B-shaped layer, 4 weights in the tile
+    layout, at M = 2048)."""
+    import torch
+    import int8_weight_quantized_w4_b200 as w4
+    dev = torch.device("cuda", 0)
+    lib = w4.lib()
+    hs = int(torch.cuda.current_stream().cuda_stream)
+    if name in ("body", "prefill-gpt2", "prefill-3p8b"):
+        shapes = synth.gpt2_stack_shapes() if name != "prefill-3p8b" else synth.dense38_stack_shapes()[:4]
+        M = {"body": 1, "prefill-gpt2": synth.GPT2_PROMPT, "prefill-3p8b": 2048}[name]
+        items = []
+        for i, (_, K, N) in enumerate(shapes):
+            W = synth.w4_weight(K, N, i)
+            qw, sc, zp = (torch.from_numpy(W[k]).to(dev) for k in ("qw", "scales", "zp"))
+            rep = w4.w4_repack if name == "body" else w4.w4t_repack
+            items.append({"x": torch.from_numpy(synth.activations(M, K, i)).to(dev), "wr": rep(qw, sc, zp, K, N),
+                          "y": torch.empty((M, N), device=dev), "K": K, "N": N})
+        descs = w4.make_rdescs(items)
+        if name == "body":
+            run = lambda: _ok(lib.w4r_matmul_grouped(descs, len(descs), hs), lib, "w4r")
+        else:
+            scratch = torch.empty(max(w4.w4t_workspace_size(descs), 16), dtype=torch.uint8, device=dev)
+            run = lambda: _ok(lib.w4t_matmul_grouped(descs, len(descs), scratch.data_ptr(), scratch.numel(), hs), lib,
+                              "w4t")
+    elif name == "head":
+        H = synth.i8_head(HEAD_K, HEAD_V)
+        tr = w4.i8_head_repack(torch.from_numpy(H["table"]).to(dev), torch.from_numpy(H["scales"]).to(dev),
+                               HEAD_K, HEAD_V)
+        h = torch.from_numpy(synth.activations(1, HEAD_K, 999)).to(dev)
+        lg = torch.empty((1, HEAD_V), device=dev)
+        run = lambda: _ok(lib.i8r_head_logits(h.data_ptr(), tr.data_ptr(), HEAD_K, HEAD_V, lg.data_ptr(), hs), lib,
+                          "i8r")
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    torch.cuda.synchronize()
+    for _ in range(calls):
+        run()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, "calls": calls}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -938,7 +984,13 @@ def main():
                     help="device seconds of the timed step replays (the body and head alone get half each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config measurements (configs 0, 2, 3, 4)")
+    ap.add_argument("--profile-case", choices=["body", "head", "prefill-gpt2", "prefill-3p8b"], default=None,
+                    help="only run one workload's kernels a few times, for a profiler (see profiles/)")
+    ap.add_argument("--calls", type=int, default=4, help="calls of --profile-case")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case, args.calls)
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
