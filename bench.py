@@ -234,8 +234,9 @@ class Workload:
             t = table if r == 0 else table.clone()
             s = hsc if r == 0 else hsc.clone()
             tr = w4.i8_head_repack(t, s, HEAD_K, HEAD_V)  # the head in its streaming layout (once, at load)
+            tt = w4.i8t_head_repack(t, s, HEAD_K, HEAD_V)  # and in the tensor cores' tile layout
             # the descriptors hold raw pointers: keep every tensor they name alive
-            self.copies.append((descs, t, s, ws, rdescs, wrs, tr))
+            self.copies.append((descs, t, s, ws, rdescs, wrs, tr, tt))
         need = max(w4.w4_matmul_grouped_workspace_size(self.copies[0][0]),
                    w4.i8_head_workspace_size(1, HEAD_K, HEAD_V))
         self.ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
@@ -264,6 +265,14 @@ class Workload:
                                       stream_handle)
         if st != 0:
             raise RuntimeError(f"i8r_head_logits failed: {st} {self.lib.w4_last_error()}")
+
+    def head_tile(self, r: int, stream_handle: int):
+        """The int8 head on the tensor cores (tile layout, integer MMAs)."""
+        tt = self.copies[r][7]
+        st = self.lib.i8t_head_logits(self.h.data_ptr(), HEAD_K, tt.data_ptr(), HEAD_K, HEAD_V, 1,
+                                      self.logits.data_ptr(), HEAD_V, stream_handle)
+        if st != 0:
+            raise RuntimeError(f"i8t_head_logits failed: {st} {self.lib.w4_last_error()}")
 
     def head_page_format(self, r: int, stream_handle: int):
         _, t, s = self.copies[r][:3]
@@ -342,11 +351,15 @@ def run_ours(args, world, rank, local):
     g_head = capture([wl.head])
     g_page = capture([wl.body_page_format])
     g_hpage = capture([wl.head_page_format])
+    g_htile = capture([wl.head_tile])
+    g_step_t = capture([wl.body, wl.head_tile])
     n_step = reps_for(g_step, args.seconds)
     n_body = reps_for(g_body, args.seconds / 2)
     n_head = reps_for(g_head, args.seconds / 2)
     n_page = reps_for(g_page, args.seconds / 4)
     n_hpage = reps_for(g_hpage, args.seconds / 4)
+    n_htile = reps_for(g_htile, args.seconds / 4)
+    n_step_t = reps_for(g_step_t, args.seconds / 4)
     sampler = ClockSampler(gpu_id(local if world > 1 else 0))
     sampler.start()
     time.sleep(0.2)
@@ -355,10 +368,12 @@ def run_ours(args, world, rank, local):
     head_avg = timed(g_head, n_head) / (K * n_head)
     page_avg = timed(g_page, n_page) / (K * n_page)
     hpage_avg = timed(g_hpage, n_hpage) / (K * n_hpage)
+    htile_avg = timed(g_htile, n_htile) / (K * n_htile)
+    step_t_avg = timed(g_step_t, n_step_t) / (K * n_step_t)
     clocks = sampler.stop()
     steps_timed = K * n_step
     ms_step = total_ms / steps_timed
-    del g_step, g_body, g_head, g_page, g_hpage
+    del g_step, g_body, g_head, g_page, g_hpage, g_htile, g_step_t
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(wl, args, world, R)
@@ -407,6 +422,10 @@ def run_ours(args, world, rank, local):
                       "GB_per_s": round(head_bytes() / (head_avg * 1e-3) / 1e9, 1),
                       "frac_of_hbm": round(head_bytes() / (head_avg * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                       "traffic": profiled_traffic("i8r_head_gpt2_m1.md")},
+        "head_tile": {"ms": round(htile_avg, 5), "kernel": "i8t_head_kernel<16> (tile layout, tcgen05 kind::i8)",
+                      "GB_per_s": round(head_bytes() / (htile_avg * 1e-3) / 1e9, 1),
+                      "frac_of_hbm": round(head_bytes() / (htile_avg * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                      "step_ms_with_it": round(step_t_avg, 5)},
         "head_page_format": {"ms": round(hpage_avg, 5),
                              "GB_per_s": round(head_bytes() / (hpage_avg * 1e-3) / 1e9, 1),
                              "kernel": "i8_rows_kernel<1> (page-format table)"},
@@ -583,7 +602,9 @@ def config0(peaks, budget):
 
 
 def config2(peaks, budget):
-    """int8 tied head [768, 50257], last position: M = 1 (streaming layout) and M = 8 (page format)."""
+    """int8 tied head [768, 50257], last position: M = 1 (streaming layout and
+    tile layout) and M = 8 (tile layout, tensor cores; the page-format
+    stream-K kernel beside it)."""
     import torch
     import int8_weight_quantized_w4_b200 as w4
     import oracle
@@ -592,8 +613,10 @@ def config2(peaks, budget):
     dev = torch.device("cuda")
     t0_, s0_ = torch.from_numpy(H["table"]).to(dev), torch.from_numpy(H["scales"]).to(dev)
     tr0 = w4.i8_head_repack(t0_, s0_, K, V)
+    tt0 = w4.i8t_head_repack(t0_, s0_, K, V)
     R = max(2, -(-3 * torch.cuda.get_device_properties(0).L2_cache_size // tr0.numel()) + 1)
     trs = [tr0] + [tr0.clone() for _ in range(R - 1)]
+    tts = [tt0] + [tt0.clone() for _ in range(R - 1)]
     tabs = [(t0_, s0_)] + [(t0_.clone(), s0_.clone()) for _ in range(R - 1)]
     lib = w4.lib()
     nbytes = synth.i8_head_bytes(K, V)
@@ -604,30 +627,43 @@ def config2(peaks, budget):
                                  "i8r_head_logits") for t in trs]
     ms1 = graph_ms(calls, 20)
     g1 = nbytes / (ms1 * 1e-3) / 1e9
+
+    def tile_calls(h, lg, M):
+        return [lambda hs, t=t: _ok(lib.i8t_head_logits(h.data_ptr(), K, t.data_ptr(), K, V, M, lg.data_ptr(), V,
+                                                        hs), lib, "i8t_head_logits") for t in tts]
+
+    ms1t = graph_ms(tile_calls(h1, lg1, 1), 20)
+    g1t = nbytes / (ms1t * 1e-3) / 1e9
     M8 = 8
     h8 = torch.from_numpy(synth.activations(M8, K, 998)).to(dev)
     lg8 = torch.empty((M8, V), device=dev)
+    ms8 = graph_ms(tile_calls(h8, lg8, M8), 20)
+    g8 = nbytes / (ms8 * 1e-3) / 1e9
     wsb = w4.i8_head_workspace_size(M8, K, V)
     ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)
     calls8 = [lambda hs, t=t, s=s_: _ok(lib.i8_head_logits(h8.data_ptr(), K, t.data_ptr(), V, s.data_ptr(),
                                                              lg8.data_ptr(), V, M8, K, V, ws.data_ptr(), ws.numel(),
                                                              hs), lib, "i8_head_logits")
               for t, s_ in tabs]
-    ms8 = graph_ms(calls8, 10)
-    g8 = nbytes / (ms8 * 1e-3) / 1e9
+    ms8p = graph_ms(calls8, 5)
     hh1, hh8 = synth.activations(1, K, 999), synth.activations(M8, K, 998)
     r1, n1, e1 = _oracle_rate(lambda: oracle.i8_head_ref(hh1, H["table"], H["scales"], K, V), nbytes / 1e9, budget / 2)
     r8, n8, e8 = _oracle_rate(lambda: oracle.i8_head_ref(hh8, H["table"], H["scales"], K, V), nbytes / 1e9, budget / 2)
-    fl8 = 2 * M8 * K * V / (ms8 * 1e-3) / 1e12
     out["M1"] = {"metric": "weight GB/s", "value": round(g1, 1), "unit": "GB/s", "us_per_call": round(ms1 * 1e3, 3),
-                 "roofline": {"kernel": "i8r_head_kernel", "bound": "hbm", "achieved": round(g1, 1),
-                              "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(g1 / peaks["hbm_gbs"], 4)},
+                 "roofline": {"kernel": "i8r_head_kernel (streaming layout)", "bound": "hbm",
+                              "achieved": round(g1, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": round(g1 / peaks["hbm_gbs"], 4)},
+                 "tile_layout": {"us_per_call": round(ms1t * 1e3, 3), "GB_per_s": round(g1t, 1),
+                                 "frac": round(g1t / peaks["hbm_gbs"], 4),
+                                 "kernel": "i8t_head_kernel<16> (tcgen05 kind::i8)"},
                  "cpu_baseline": _cpu(round(r1, 4), "GB/s", "oracle i8_head_ref, M=1", n1, e1)}
     out["M8"] = {"metric": "weight GB/s", "value": round(g8, 1), "unit": "GB/s", "us_per_call": round(ms8 * 1e3, 3),
-                 "roofline": {"kernel": "i8_head_kernel<8> (page format, stream-K)", "bound": "hbm",
+                 "roofline": {"kernel": "i8t_head_kernel<64> (tile layout, tcgen05 kind::i8, N 64)", "bound": "hbm",
                               "achieved": round(g8, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                              "frac": round(g8 / peaks["hbm_gbs"], 4),
-                              "fp32_tflops": round(fl8, 2)},
+                              "frac": round(g8 / peaks["hbm_gbs"], 4)},
+                 "page_format": {"us_per_call": round(ms8p * 1e3, 3),
+                                 "GB_per_s": round(nbytes / (ms8p * 1e-3) / 1e9, 1),
+                                 "kernel": "i8_head_kernel<8> (page format, stream-K, fp32 FMA)"},
                  "cpu_baseline": _cpu(round(r8, 4), "GB/s", "oracle i8_head_ref, M=8", n8, e8)}
     return out
 

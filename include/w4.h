@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define W4_ABI_VERSION 3
+#define W4_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define W4_API __attribute__((visibility("default")))
@@ -389,6 +389,58 @@ W4_API w4_status i8r_head_logits(const float* h, const void* tr, int64_t K, int6
  * 8 bytes of device memory (8-byte aligned) that the call clears and uses. */
 W4_API w4_status i8r_head_argmax(const float* h, const void* tr, int64_t K, int64_t V, int32_t* token,
                                  float* best_logit, void* keys, void* stream);
+
+/* The tile layout of the int8 head, read by the tensor-core head
+ * (i8t_head_logits / i8t_head_argmax) for 1 to 8 last-position rows. The
+ * page's table bytes and scales ("ONNX export, quantization and the browser
+ * runtime", section "Quantization (train/quantize.py)", step 3) reordered
+ * once at load time into the tensor core's int8 operand layout; nothing is
+ * changed or rounded: i8t_head_repack_restore gives back the page's table
+ * and scales exactly.
+ *
+ * Layout, K % 32 == 0, 32 <= K <= 1024: tiles of 128 tokens in token order,
+ * each K / 32 units of 4096 bytes and then the tile's 128 scales (fp32). In
+ * unit u of tile t the code of row 32 u + 16 h + i (h in 0..1, i in 0..15)
+ * and token 128 t + c sits at byte (c / 8) * 256 + h * 128 + (c % 8) * 16 + i;
+ * the scale of token 128 t + c at byte K * 128 + 4 c of the tile. Tokens at
+ * or past V hold code 0 and scale 0. i8t_head_repacked_bytes() is the size
+ * (0 for a shape the layout does not take). */
+W4_API size_t i8t_head_repacked_bytes(int64_t K, int64_t V);
+
+/* Page format (table [K, V] with row stride ldt >= V, any alignment;
+ * scales [V] fp32, 4-byte aligned) -> tile layout (i8t_head_repacked_bytes
+ * bytes, 16-byte aligned), on the GPU. W4_ERR_SHAPE for a shape the layout
+ * does not take. */
+W4_API w4_status i8t_head_repack(const int8_t* table, int64_t ldt, const float* scales, int64_t K, int64_t V,
+                                 void* tiles, void* stream);
+
+/* Tile layout -> page format (the exact inverse of i8t_head_repack). */
+W4_API w4_status i8t_head_repack_restore(const void* tiles, int64_t K, int64_t V, int8_t* table, int64_t ldt,
+                                         float* scales, void* stream);
+
+/* logits[m, v] = s_v * sum_k h[m, k] T[k, v] for M <= 8 last-position rows
+ * h [M, K] (row stride ldh >= K when M > 1, 4-byte aligned) on a head in the
+ * tile layout; logits [M, V] with row stride ldl >= V when M > 1, 4-byte
+ * aligned, fully overwritten. The tensor cores multiply the codes by h
+ * written per row in fixed point (8 signed 7-bit digits against the row's
+ * largest magnitude: exact for every element within 2^31 of it, within
+ * 2^-55 of it otherwise) with exact integer sums, and the digits are weighed
+ * and scaled in fp64: each logit is the dot product rounded about once, and
+ * deterministic. A row holding an Inf or NaN gives NaN logits. No workspace.
+ * The launch may start streaming the table before the previous work on the
+ * stream has finished; h is read and the logits written only after it has.
+ * W4_ERR_SHAPE for M > 8 or a shape the layout does not take; M = 0 or
+ * V = 0 is a no-op. */
+W4_API w4_status i8t_head_logits(const float* h, int64_t ldh, const void* tiles, int64_t K, int64_t V, int64_t M,
+                                 float* logits, int64_t ldl, void* stream);
+
+/* Greedy decoding with the tensor-core head: tokens[m] = argmax_v of exactly
+ * the logits i8t_head_logits computes (ties to the lowest id; -0 equals +0),
+ * best_logits[m] (may be NULL) = that logit; the logits are not written.
+ * keys: 8 M bytes of device memory (8-byte aligned) that the call clears and
+ * uses. tokens / best_logits: M entries on the device. */
+W4_API w4_status i8t_head_argmax(const float* h, int64_t ldh, const void* tiles, int64_t K, int64_t V, int64_t M,
+                                 int32_t* tokens, float* best_logits, void* keys, void* stream);
 
 /* Greedy decoding on the head: tokens[m] = argmax_v logits[m, v] (ties to
  * the lowest token id), best_logits[m] = that logit when best_logits is not

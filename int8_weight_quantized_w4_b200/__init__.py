@@ -14,6 +14,8 @@ Operations (see include/w4.h for layouts and error behaviour):
   i8_head_logits(h, table, scales, K, V)    last-position logits, int8 head
   i8_head_repack(table, scales, K, V)       the head in the streaming layout (once, at load)
   i8r_head_logits(h, tr, K, V) / _argmax    M = 1 head on the repacked table
+  i8t_head_repack(table, scales, K, V)      the head in the tensor cores' tile layout (once, at load)
+  i8t_head_logits(h, tiles, K, V) / _argmax M <= 8 rows on the tensor-core head
   w4_quantize(w, block, scale_type)         the dq4 quantiser (GPU)
   i8_quantize_head(w)                       the embedding_int8 quantiser (GPU)
   pack_nibbles / unpack_nibbles             host-side UINT4 packing
@@ -406,6 +408,59 @@ def i8r_head_argmax(h, tr, K: int, V: int, stream=None):
     keys = torch.empty(1, dtype=torch.int64, device=h.device)
     _check(lib().i8r_head_argmax(_ptr(h), _ptr(tr), K, V, _ptr(tok), _ptr(best), _ptr(keys), _stream_handle(stream)),
            "i8r_head_argmax")
+    return tok, best
+
+
+def i8t_head_repacked_bytes(K: int, V: int) -> int:
+    return int(lib().i8t_head_repacked_bytes(K, V))
+
+
+def i8t_head_repack(table, scales, K: int, V: int, ldt: int | None = None, stream=None):
+    """The int8 head (page format) in the tile layout the tensor-core head
+    reads: a uint8 device tensor of i8t_head_repacked_bytes(K, V) bytes."""
+    torch = _torch()
+    ldt = V if ldt is None else ldt
+    n = i8t_head_repacked_bytes(K, V)
+    if n == 0:
+        raise ValueError(f"the head tile layout does not take K={K}, V={V}")
+    out = torch.empty(n, dtype=torch.uint8, device=table.device)
+    _check(lib().i8t_head_repack(_ptr(table), ldt, _ptr(scales), K, V, _ptr(out), _stream_handle(stream)),
+           "i8t_head_repack")
+    return out
+
+
+def i8t_head_repack_restore(tiles, K: int, V: int, stream=None):
+    """(table [K, V] int8, scales [V] fp32) of a head in the tile layout."""
+    torch = _torch()
+    table = torch.empty((K, V), dtype=torch.int8, device=tiles.device)
+    sc = torch.empty(V, dtype=torch.float32, device=tiles.device)
+    _check(lib().i8t_head_repack_restore(_ptr(tiles), K, V, _ptr(table), V, _ptr(sc), _stream_handle(stream)),
+           "i8t_head_repack_restore")
+    return table, sc
+
+
+def i8t_head_logits(h, tiles, K: int, V: int, logits=None, stream=None):
+    """logits [M, V] of M <= 8 last-position rows h [M, K] on the tensor-core
+    head (tile layout)."""
+    torch = _torch()
+    M = h.shape[0] if h.dim() == 2 else 1
+    if logits is None:
+        logits = torch.empty((M, V), dtype=torch.float32, device=h.device)
+    _check(lib().i8t_head_logits(_ptr(h), _ld(h, K), _ptr(tiles), K, V, M, _ptr(logits), _ld(logits, V),
+                                 _stream_handle(stream)), "i8t_head_logits")
+    return logits
+
+
+def i8t_head_argmax(h, tiles, K: int, V: int, stream=None):
+    """(tokens int32 [M], best logits fp32 [M]) of M <= 8 rows h on the
+    tensor-core head."""
+    torch = _torch()
+    M = h.shape[0] if h.dim() == 2 else 1
+    tok = torch.empty(M, dtype=torch.int32, device=h.device)
+    best = torch.empty(M, dtype=torch.float32, device=h.device)
+    keys = torch.empty(max(M, 1), dtype=torch.int64, device=h.device)
+    _check(lib().i8t_head_argmax(_ptr(h), _ld(h, K), _ptr(tiles), K, V, M, _ptr(tok), _ptr(best), _ptr(keys),
+                                 _stream_handle(stream)), "i8t_head_argmax")
     return tok, best
 
 

@@ -13,8 +13,10 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 @pytest.mark.parametrize("summary,algorithmic", [
-    ("w4_gemv_gpt2_m1.md", bench.body_bytes()),
-    ("i8_rows_gpt2_head_m1.md", bench.head_bytes()),
+    ("w4r_gemv_gpt2_m1.md", bench.body_bytes()),
+    ("i8r_head_gpt2_m1.md", bench.head_bytes()),
+    ("w4_gemv_pageformat_gpt2_m1.md", bench.body_bytes()),
+    ("i8_rows_pageformat_gpt2_head_m1.md", bench.head_bytes()),
 ])
 def test_committed_profiles_are_machine_readable(summary, algorithmic):
     """Each summary names its kernel's source, a 16-hex-digit hash and the
