@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define W4_ABI_VERSION 4
+#define W4_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define W4_API __attribute__((visibility("default")))
@@ -320,6 +320,33 @@ W4_API size_t w4t_workspace_size(const w4t_desc* descs, int32_t count);
 W4_API w4_status w4t_matmul_grouped(const w4t_desc* descs, int32_t count, void* workspace, size_t workspace_bytes,
                                     void* stream);
 W4_API w4_status w4t_matmul(const w4t_desc* d, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Decode matmuls (one row of x) on weights in the tile layout, on the tensor
+ * cores with integer MMAs: y[1, N] = act(x[1, K] . W + bias) + residual.
+ * x is written in fixed point against its largest magnitude, as 8 signed
+ * 7-bit digits per element (exact for every element within 2^31 of the
+ * largest, within 2^-55 of it otherwise); the MMA multiplies the digits by
+ * the stored codes q exactly in int32, the zero point enters exactly as
+ * D - zp * (block sum of the digits), and each block's integer sums are
+ * weighed and scaled by s in fp32 and summed over the blocks in fp32.
+ * Non-finite x give NaN.
+ * - descs: HOST array of w4t_desc (wr = the tile-layout weight), read during
+ *   the call only. M must be 1 (0 skips the descriptor), K % 32 == 0,
+ *   K <= 3072, N % 8 == 0; x / y / bias / residual 4-byte aligned, wr
+ *   16-byte aligned; ldx / ldy / ldr are not used. K = 0 writes the
+ *   epilogue of 0. Outputs must not overlap each other or any input.
+ * - workspace: device memory of at least w4i_workspace_size(descs, count)
+ *   bytes (about 8.5 K per distinct x), 16-byte aligned; it receives the
+ *   digits of each distinct x and needs no zeroing. Calls that may run at the
+ *   same time must not share it.
+ * - The digits are written by one launch, then the GEMV runs (a second
+ *   launch); both start early on the stream (programmatic dependent launch)
+ *   and read x, bias and the residual and write y only after the previous
+ *   work on the stream has completed. */
+W4_API size_t w4i_workspace_size(const w4t_desc* descs, int32_t count);
+W4_API w4_status w4i_matmul_grouped(const w4t_desc* descs, int32_t count, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+W4_API w4_status w4i_matmul(const w4t_desc* d, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------ head */
 

@@ -14,6 +14,7 @@ Operations (see include/w4.h for layouts and error behaviour):
   i8_head_logits(h, table, scales, K, V)    last-position logits, int8 head
   i8_head_repack(table, scales, K, V)       the head in the streaming layout (once, at load)
   i8r_head_logits(h, tr, K, V) / _argmax    M = 1 head on the repacked table
+  w4i_matmul(x, wt, K, N)                   M = 1 on the tile layout: integer tensor-core MMAs
   i8t_head_repack(table, scales, K, V)      the head in the tensor cores' tile layout (once, at load)
   i8t_head_logits(h, tiles, K, V) / _argmax M <= 8 rows on the tensor-core head
   w4_quantize(w, block, scale_type)         the dq4 quantiser (GPU)
@@ -319,6 +320,36 @@ def w4t_matmul(x, wt, K: int, N: int, y=None, ws=None, stream=None, bias=None, r
         y = torch.empty((x.shape[0], N), dtype=torch.float32, device=x.device)
     item = {"x": x, "wr": wt, "y": y, "K": K, "N": N, "bias": bias, "residual": residual, "act": act}
     w4t_matmul_grouped(descs=make_rdescs([item]), ws=ws, stream=stream)
+    return y
+
+
+def w4i_workspace_size(descs) -> int:
+    return int(lib().w4i_workspace_size(descs, len(descs)))
+
+
+def w4i_matmul_grouped(items: Sequence[dict] | None = None, descs=None, ws=None, stream=None):
+    """Decode matmuls (M = 1) on tile-layout weights ("wr" = w4t_repack output)
+    with integer tensor-core MMAs; items as for make_rdescs (x [1, K])."""
+    if descs is None:
+        descs = make_rdescs(items)
+    need = w4i_workspace_size(descs)
+    if ws is None:
+        ws = tile_workspace(need)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().w4i_matmul_grouped(descs, len(descs), _ptr(ws), nbytes, _stream_handle(stream)),
+           "w4i_matmul_grouped")
+
+
+def w4i_matmul(x, wt, K: int, N: int, y=None, ws=None, stream=None, bias=None, residual=None, act: str = "none"):
+    """y[1, N] = act(x[1, K] . W + bias) + residual with W in the tile layout
+    (w4t_repack), on the integer tensor-core GEMV; returns y."""
+    torch = _torch()
+    if x.dim() == 1:
+        x = x.view(1, -1)
+    if y is None:
+        y = torch.empty((x.shape[0], N), dtype=torch.float32, device=x.device)
+    item = {"x": x, "wr": wt, "y": y, "K": K, "N": N, "bias": bias, "residual": residual, "act": act}
+    w4i_matmul_grouped(descs=make_rdescs([item]), ws=ws, stream=stream)
     return y
 
 

@@ -27,7 +27,7 @@ W4_OK, W4_ERR_NULL, W4_ERR_SHAPE, W4_ERR_ALIGN, W4_ERR_DEVICE, W4_ERR_CUDA, W4_E
     W4_ERR_VALUE = range(9)
 PATHS = {"auto": 0, "gemv": 1, "generic": 2, "tc": 3}
 ACTS = {"none": 0, "gelu_tanh": 1, "gelu_erf": 2}
-ABI_VERSION = 4
+ABI_VERSION = 5
 GROUP_MAX = 48
 
 
@@ -94,6 +94,9 @@ SIGNATURES = {
     "w4t_workspace_size": (C.c_size_t, [C.POINTER(W4RDesc), C.c_int32]),
     "w4t_matmul_grouped": (C.c_int, [C.POINTER(W4RDesc), C.c_int32, C.c_void_p, C.c_size_t, C.c_void_p]),
     "w4t_matmul": (C.c_int, [C.POINTER(W4RDesc), C.c_void_p, C.c_size_t, C.c_void_p]),
+    "w4i_workspace_size": (C.c_size_t, [C.POINTER(W4RDesc), C.c_int32]),
+    "w4i_matmul_grouped": (C.c_int, [C.POINTER(W4RDesc), C.c_int32, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "w4i_matmul": (C.c_int, [C.POINTER(W4RDesc), C.c_void_p, C.c_size_t, C.c_void_p]),
     "w4r_matmul_grouped": (C.c_int, [C.POINTER(W4RDesc), C.c_int32, C.c_void_p]),
     "i8_head_repacked_bytes": (C.c_size_t, [C.c_int64, C.c_int64]),
     "i8_head_repack": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),

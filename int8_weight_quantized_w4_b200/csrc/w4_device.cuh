@@ -23,7 +23,7 @@ struct ErrorWord {
   int32_t detail;
 };
 
-enum KernelId : int32_t { K_GEMV = 1, K_GENERIC = 2, K_HEAD = 3, K_HEAD_GENERIC = 4, K_TC = 5, K_EMBED = 6, K_GEMVR = 7, K_HEADR = 8, K_DEBUG = 9, K_TILE = 10, K_HEADT = 11 };
+enum KernelId : int32_t { K_GEMV = 1, K_GENERIC = 2, K_HEAD = 3, K_HEAD_GENERIC = 4, K_TC = 5, K_EMBED = 6, K_GEMVR = 7, K_HEADR = 8, K_DEBUG = 9, K_TILE = 10, K_HEADT = 11, K_GEMVI = 12 };
 
 __device__ __forceinline__ void record_error(ErrorWord* e, int32_t status, int32_t kernel, int32_t detail) {
   if (atomicCAS(&e->status, 0, status) == 0) {
