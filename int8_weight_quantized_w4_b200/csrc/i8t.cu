@@ -40,9 +40,9 @@
 //    bulk copy, no multicast) through a ring of 10 to 13 stages; the codes do
 //    not depend on the previous launch, so the first stages are requested
 //    before it has finished;
-//  * warps 0 and 1 each issue the MMAs of every other stage of a tile (four
-//    MMAs of M 128, N 8 M rounded up to 16, K 32) into accumulators of their
-//    own in tensor memory, so that the wait of one issuing thread (an
+//  * warps 0 and 1 each issue the MMAs of every other stage (four MMAs of
+//    M 128, N 8 M rounded up to 16, K 32) into accumulators of their own in
+//    tensor memory, one per tile, so that the wait of one issuing thread (an
 //    mbarrier wait right after MMAs costs it a few hundred clocks) overlaps
 //    the other's MMAs. The MMA's commit frees the stage for the next copy;
 //  * warps 4-7 (one per quarter of tensor-memory lanes, a lane per token)
@@ -81,8 +81,9 @@ constexpr int SMEM_MAX = 227 * 1024;
 constexpr int BAR_BYTES = 512;             // barriers, tensor-memory slot, abort flag, row exponents
 
 __host__ __device__ constexpr int nb_for(int M) { return M <= 2 ? 16 : (M <= 4 ? 32 : (M <= 6 ? 48 : 64)); }
+// even: the two issuers take the stages of one parity each
 __host__ __device__ constexpr int stages_for(int NB, int K) {
-  return (SMEM_MAX - NB * K - BAR_BYTES) / SB < MAXNS ? (SMEM_MAX - NB * K - BAR_BYTES) / SB : MAXNS;
+  return ((SMEM_MAX - NB * K - BAR_BYTES) / SB < MAXNS ? (SMEM_MAX - NB * K - BAR_BYTES) / SB : MAXNS) & ~1;
 }
 __host__ __device__ constexpr int smem_for(int NB, int K) { return stages_for(NB, K) * SB + NB * K + BAR_BYTES; }
 static_assert(stages_for(64, KMAX) >= 8, "stage ring of the widest case");
@@ -373,54 +374,62 @@ __global__ void __launch_bounds__(NT, 1) i8t_head_kernel(const __grid_constant__
       const uint64_t adesc0 = sdesc(smem_u32(stages));
       const uint64_t bdesc0 = sdesc(smem_u32(bs));
       const int tail = upt - SU * (nst - 1);  // units of the last stage of a tile
-      int s = X;                              // ring slot of the next stage
+      // The CTA's stages g = X, X + 2, ... (every stage when issuer 1 is idle);
+      // stage g is stage j = g % nst of tile g / nst. With the ring's even size
+      // a ring slot always serves the same issuer, which so sees every phase
+      // of its barrier in order.
+      const int step = two ? 2 : 1;
+      int g = two ? X : 0, ti = 0, j = g;  // j < nst: issuer 1 runs only when nst >= 2
+      int s = g;                           // ring slot of stage g (g < NS)
       uint32_t ph = 0;
-      if (s >= NS) {
-        s -= NS;
-        ph = 1u;
-      }
-      int last = -1;  // last tile whose accumulator was committed
-      bool ok = true;
+      int cur = -1;                        // the tile whose accumulator takes this issuer's MMAs
+      int s_last = -1;                     // ring slot and phase parity of the last commit to empty
+      uint32_t ph_last = 0;
+      bool first = true;
+      uint32_t dt = 0;
 #pragma unroll 1
-      for (int ti = 0; ti < t1 - t0 && ok; ++ti) {
-        const int d = ti & 1;
-        if (ti >= 2 && !spin_wait(&dfree[2 * X + d], static_cast<uint32_t>((ti >> 1) - 1) & 1u, budget, abort_flag,
-                                  p.err, 2))
-          break;
-        const uint32_t dt = tmem + static_cast<uint32_t>((2 * X + d) * NB);
-#pragma unroll 1
-        for (int j = X; j < nst; j += 2) {
-          if (!spin_wait(&full[s], ph, budget, abort_flag, p.err, 3)) {
-            ok = false;
+      while (g < GS) {
+        if (ti != cur) {
+          if (cur >= 0) mma_commit(&dready[2 * X + (cur & 1)]);
+          cur = ti;
+          const int d = ti & 1;
+          if (ti >= 2 && !spin_wait(&dfree[2 * X + d], static_cast<uint32_t>((ti >> 1) - 1) & 1u, budget, abort_flag,
+                                    p.err, 2))
             break;
-          }
-          tc_fence_after();
-          const uint64_t ad = adesc0 + static_cast<uint64_t>(s) * (SB >> 4);
-          const uint64_t bd = bdesc0 + static_cast<uint64_t>(j) * (SU * BSTEP);
-          if (j < nst - 1 || tail == SU) {
-            mma_i8(dt, ad, bd, IDESC, j != X);
-            mma_i8(dt, ad + ASTEP, bd + BSTEP, IDESC, true);
-            mma_i8(dt, ad + 2 * ASTEP, bd + 2 * BSTEP, IDESC, true);
-            mma_i8(dt, ad + 3 * ASTEP, bd + 3 * BSTEP, IDESC, true);
-          } else {
-            for (int q = 0; q < tail; ++q)
-              mma_i8(dt, ad + q * ASTEP, bd + q * BSTEP, IDESC, j != X || q != 0);
-          }
-          mma_commit(&empty[s]);
-          // next stage of this issuer: two on, or the first of the next tile
-          const int step = j + 2 < nst ? 2 : nst - j + X;
-          s += step;
-          while (s >= NS) {
-            s -= NS;
-            ph ^= 1u;
-          }
+          dt = tmem + static_cast<uint32_t>((2 * X + d) * NB);
+          first = true;
         }
-        if (!ok) break;
-        mma_commit(&dready[2 * X + d]);
-        last = ti;
+        if (!spin_wait(&full[s], ph, budget, abort_flag, p.err, 3)) break;
+        tc_fence_after();
+        const uint64_t ad = adesc0 + static_cast<uint64_t>(s) * (SB >> 4);
+        const uint64_t bd = bdesc0 + static_cast<uint64_t>(j) * (SU * BSTEP);
+        if (j < nst - 1 || tail == SU) {
+          mma_i8(dt, ad, bd, IDESC, !first);
+          mma_i8(dt, ad + ASTEP, bd + BSTEP, IDESC, true);
+          mma_i8(dt, ad + 2 * ASTEP, bd + 2 * BSTEP, IDESC, true);
+          mma_i8(dt, ad + 3 * ASTEP, bd + 3 * BSTEP, IDESC, true);
+        } else {
+          for (int q = 0; q < tail; ++q) mma_i8(dt, ad + q * ASTEP, bd + q * BSTEP, IDESC, !first || q != 0);
+        }
+        first = false;
+        mma_commit(&empty[s]);
+        s_last = s;
+        ph_last = ph;
+        g += step;
+        j += step;
+        while (j >= nst) {
+          j -= nst;
+          ++ti;
+        }
+        s += step;
+        if (s >= NS) {
+          s -= NS;
+          ph ^= 1u;
+        }
       }
-      // the last commit covers every MMA issued before it
-      if (last >= 0) mbar_wait_drain(&dready[2 * X + (last & 1)], static_cast<uint32_t>(last >> 1) & 1u, p.timeout_ns);
+      if (g >= GS && cur >= 0) mma_commit(&dready[2 * X + (cur & 1)]);
+      // the last commit to empty covers every MMA of this thread
+      if (s_last >= 0) mbar_wait_drain(&empty[s_last], ph_last, p.timeout_ns);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ read back (warps 4-7)

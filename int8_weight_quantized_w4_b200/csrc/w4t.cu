@@ -101,16 +101,22 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
 // bytes of one block of one row tile of pieces, and of one stage
 __host__ __device__ constexpr int piece_bytes(int nx) { return 192 * nx; }
 __host__ __device__ constexpr int stage_bytes(int nx) { return (192 * nx + BLK + 127) / 128 * 128; }
+// Both rings have an even number of entries: the issuers, and with eight
+// decode warps the decode pairs, take the blocks of one parity each, so a
+// ring entry then always serves the same waiters, which see every phase of
+// its barriers in order (a parity wait one phase ahead of a phase its waiter
+// has not seen complete would pass spuriously).
 __host__ __device__ constexpr int ring_stages(int nx) {
-  return RING / stage_bytes(nx) < MAXST ? RING / stage_bytes(nx) : MAXST;
+  return (RING / stage_bytes(nx) < MAXST ? RING / stage_bytes(nx) : MAXST) & ~1;
 }
 // Slots of tensor memory (an accumulator of NX columns and an A operand of
-// 16): as many as 512 columns hold, at most MAXSLOT (3 for NX = 128, 6 for 64,
-// 8 below). A block's slot is busy from its decode to its read-back, so more
-// slots keep more blocks between the two.
+// 16): as many as 512 columns hold, at most MAXSLOT, even (2 for NX = 128, 6
+// for 64, 8 below). A block's slot is busy from its decode to its read-back,
+// so more slots keep more blocks between the two.
 __host__ __device__ constexpr int tmem_slots(int nx) {
-  return static_cast<int>(TCOLS) / (nx + 16) < MAXSLOT ? static_cast<int>(TCOLS) / (nx + 16) : MAXSLOT;
+  return (static_cast<int>(TCOLS) / (nx + 16) < MAXSLOT ? static_cast<int>(TCOLS) / (nx + 16) : MAXSLOT) & ~1;
 }
+static_assert(ring_stages(128) >= 4 && tmem_slots(128) >= 2, "rings of the widest row tile");
 
 struct TMat {
   const uint8_t* wt;  // tile layout
