@@ -425,6 +425,7 @@ def run_ours(args, world, rank, local):
         "head_tile": {"ms": round(htile_avg, 5), "kernel": "i8t_head_kernel<16> (tile layout, tcgen05 kind::i8)",
                       "GB_per_s": round(head_bytes() / (htile_avg * 1e-3) / 1e9, 1),
                       "frac_of_hbm": round(head_bytes() / (htile_avg * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                      "traffic": profiled_traffic("i8t_head_gpt2_m1.md"),
                       "step_ms_with_it": round(step_t_avg, 5)},
         "head_page_format": {"ms": round(hpage_avg, 5),
                              "GB_per_s": round(head_bytes() / (hpage_avg * 1e-3) / 1e9, 1),
@@ -660,7 +661,8 @@ def config2(peaks, budget):
     out["M8"] = {"metric": "weight GB/s", "value": round(g8, 1), "unit": "GB/s", "us_per_call": round(ms8 * 1e3, 3),
                  "roofline": {"kernel": "i8t_head_kernel<64> (tile layout, tcgen05 kind::i8, N 64)", "bound": "hbm",
                               "achieved": round(g8, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                              "frac": round(g8 / peaks["hbm_gbs"], 4)},
+                              "frac": round(g8 / peaks["hbm_gbs"], 4),
+                              "traffic": profiled_traffic("i8t_head_gpt2_m8.md")},
                  "page_format": {"us_per_call": round(ms8p * 1e3, 3),
                                  "GB_per_s": round(nbytes / (ms8p * 1e-3) / 1e9, 1),
                                  "kernel": "i8_head_kernel<8> (page format, stream-K, fp32 FMA)"},
@@ -967,7 +969,8 @@ def profile_case(name: str, calls: int) -> None:
     """Run one workload's kernels `calls` times (no timing, no output but one
     line) so that a profiler can capture them: "body" (the 48 GPT-2 weights
     in the streaming layout, M = 1), "head" (the int8 head, streaming
-    layout, M = 1), "prefill-gpt2" (the 48 weights in the tile layout at
+    layout, M = 1), "head-tile" / "head-tile-m8" (the int8 head in the tile
+    layout, tensor cores, M = 1 / 8), "prefill-gpt2" (the 48 weights in the tile layout at
     M = 58), "prefill-3p8b" (one 3.8B-shaped layer, 4 weights in the tile
     layout, at M = 2048)."""
     import torch
@@ -992,6 +995,15 @@ def profile_case(name: str, calls: int) -> None:
             scratch = torch.empty(max(w4.w4t_workspace_size(descs), 16), dtype=torch.uint8, device=dev)
             run = lambda: _ok(lib.w4t_matmul_grouped(descs, len(descs), scratch.data_ptr(), scratch.numel(), hs), lib,
                               "w4t")
+    elif name in ("head-tile", "head-tile-m8"):
+        H = synth.i8_head(HEAD_K, HEAD_V)
+        tt = w4.i8t_head_repack(torch.from_numpy(H["table"]).to(dev), torch.from_numpy(H["scales"]).to(dev),
+                                HEAD_K, HEAD_V)
+        M = 8 if name == "head-tile-m8" else 1
+        h = torch.from_numpy(synth.activations(M, HEAD_K, 998)).to(dev)
+        lg = torch.empty((M, HEAD_V), device=dev)
+        run = lambda: _ok(lib.i8t_head_logits(h.data_ptr(), HEAD_K, tt.data_ptr(), HEAD_K, HEAD_V, M, lg.data_ptr(),
+                                              HEAD_V, hs), lib, "i8t")
     elif name == "head":
         H = synth.i8_head(HEAD_K, HEAD_V)
         tr = w4.i8_head_repack(torch.from_numpy(H["table"]).to(dev), torch.from_numpy(H["scales"]).to(dev),
@@ -1020,7 +1032,8 @@ def main():
                     help="device seconds of the timed step replays (the body and head alone get half each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config measurements (configs 0, 2, 3, 4)")
-    ap.add_argument("--profile-case", choices=["body", "head", "prefill-gpt2", "prefill-3p8b"], default=None,
+    ap.add_argument("--profile-case", choices=["body", "head", "head-tile", "head-tile-m8", "prefill-gpt2", "prefill-3p8b"],
+                    default=None,
                     help="only run one workload's kernels a few times, for a profiler (see profiles/)")
     ap.add_argument("--calls", type=int, default=4, help="calls of --profile-case")
     args = ap.parse_args()

@@ -17,6 +17,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     ("i8r_head_gpt2_m1.md", bench.head_bytes()),
     ("w4_gemv_pageformat_gpt2_m1.md", bench.body_bytes()),
     ("i8_rows_pageformat_gpt2_head_m1.md", bench.head_bytes()),
+    ("i8t_head_gpt2_m1.md", bench.head_bytes()),
+    ("i8t_head_gpt2_m8.md", bench.head_bytes()),
 ])
 def test_committed_profiles_are_machine_readable(summary, algorithmic):
     """Each summary names its kernel's source, a 16-hex-digit hash and the
