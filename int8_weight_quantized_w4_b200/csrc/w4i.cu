@@ -28,18 +28,21 @@
 //    the block sums Z_pb and 2^(E - 13) into the caller's workspace.
 //  * w4i_gemv_kernel: one persistent CTA per SM over a list of 128-column
 //    tiles the host deals out largest first. The MMA's M = 128 are the
-//    tile's columns (operand A: the codes as bytes, shared memory), N = 16
+//    tile's columns (operand A: the codes as bytes, tensor memory), N = 16
 //    its digit rows (operand B: the 8 digit rows of x and 8 rows of zeros,
 //    shared memory); each block (K = 32) has an accumulator of its own in
-//    tensor memory.
+//    tensor memory. With A out of shared memory, the weight ring takes
+//    almost all of it (14 stages, 147 KB in flight per SM).
 //    - warp 2 streams each tile's digits (one bulk copy, from L2) into one of
 //      two B slots, and the tile's blocks in groups of four (one bulk copy of
 //      up to 10496 bytes, no multicast) through a ring of stages;
 //    - warps 4-7 and 12-15, two teams of four, take the groups of one parity
-//      each (a warp one block): two logic operations per word of 8 nibbles
-//      give the codes as bytes in a fixed permutation of K, stored as the A
-//      operand, and the group's scales and zero points go to a slot of their
-//      own; then the stage goes back to the producer;
+//      each (a warp one quarter of the tile's columns, the tensor-memory
+//      lanes it may write): two logic operations per word of 8 nibbles give
+//      the codes as bytes in a fixed permutation of K, stored into tensor
+//      memory as the A operand, and the group's scales and zero points go to
+//      a slot of their own (warp j those of block j); then the stage goes
+//      back to the producer;
 //    - warps 0 and 1 take the groups of one parity each and issue their MMAs
 //      (kind::i8, M 128, N 16, K 32; one per block); one commit frees the A
 //      operand, one hands the accumulators to the read-back;
@@ -72,8 +75,6 @@ constexpr int TN = 128;                    // columns of a tile = MMA M
 constexpr int BLK = 2624;                  // bytes of one block of a tile (tile layout)
 constexpr int GB = 4;                      // blocks per group
 constexpr int GBYTES = GB * BLK;           // 10496 bytes per weight stage
-constexpr int AB = 4096;                   // A bytes of one block (128 columns x 32 codes)
-constexpr int ASLOT = GB * AB;             // 16 KB: the A operand of one group
 constexpr int SZ = 576;                    // scales and zero points of one block
 constexpr int SSLOT = GB * SZ;             // 2304 bytes: those of one group
 constexpr int KMAX = 3072;                 // rows of K this path takes
@@ -85,21 +86,24 @@ constexpr int LCAP = 4096;                 // tiles per launch
 // the groups G with G % 2 == t), so each barrier's phases are all observed,
 // in order, by the same waiters: a parity wait is never a phase ahead of a
 // phase its waiter has not seen complete (which would pass spuriously).
-constexpr int NWS = 8;                     // weight stages
+constexpr int NWS = 14;                    // weight stages
 constexpr int NA = 4;                      // A slots: free again once the group's MMAs complete
-constexpr int NS = 8;                      // scale slots and accumulator groups: free after the read-back
+constexpr int NS = 6;                      // scale slots and accumulator groups: free after the read-back
 constexpr int NWARP = 20;
 constexpr int NT = NWARP * 32;
-constexpr uint32_t TCOLS = 512;            // tensor memory: NS groups x 4 blocks x 16 columns
+// tensor memory: NS groups x 4 blocks x 16 accumulator columns, then NA
+// groups x 4 blocks x 8 columns of A (32 code bytes per lane = column)
+constexpr uint32_t TCOLS = 512;
+constexpr uint32_t TA0 = NS * GB * 16;
+static_assert(TA0 + NA * GB * 8 <= TCOLS, "tensor memory of one CTA");
 // digits buffer of one x (workspace and B slots): [K/32 x 256 digit bytes]
 // [K/32 x 4 int32: the block sums of the digits in pairs, 128 Z_2i + Z_2i+1]
 // [double 2^(E - 13)][8 bytes pad]
 __host__ __device__ constexpr int dig_bytes(int K) { return K * 8 + K / 2 + 16; }
 constexpr int BSLOT = (dig_bytes(KMAX) + 127) / 128 * 128;  // 26240
 constexpr int OFF_W = 0;
-constexpr int OFF_A = OFF_W + NWS * GBYTES;                 // 83968
-constexpr int OFF_S = OFF_A + NA * ASLOT;                   // + 65536
-constexpr int OFF_B = OFF_S + NS * SSLOT;                   // + 18432
+constexpr int OFF_S = OFF_W + NWS * GBYTES;                 // 146944
+constexpr int OFF_B = OFF_S + NS * SSLOT;                   // + 13824
 constexpr int OFF_Z = OFF_B + 2 * BSLOT;                    // + 52480: 256 zero bytes, the B rows past the digits
 constexpr int OFF_C = OFF_Z + 256;                          // the two read-back sets' partial sums of a tile:
 constexpr int CBYTES = 2 * 2 * TN * 4 + 2 * 4 * 4 * 2;      // [tile parity][set][column] + counts + sequence
@@ -107,7 +111,7 @@ constexpr int OFF_BAR = OFF_C + CBYTES;
 constexpr int NBAR = 2 * NWS + 2 * NA + 3 * NS + 4;
 constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
-static_assert(OFF_A % 128 == 0 && OFF_S % 128 == 0 && OFF_B % 128 == 0 && OFF_Z % 128 == 0 && OFF_BAR % 8 == 0,
+static_assert(OFF_S % 128 == 0 && OFF_B % 128 == 0 && OFF_Z % 128 == 0 && OFF_BAR % 8 == 0,
               "alignment");
 static_assert(NWS % 2 == 0 && NA % 2 == 0 && NS % 2 == 0, "rings pair with group parity");
 
@@ -301,13 +305,20 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t sbo) {
   return d;
 }
 
-// D (s32, tensor memory) = A (s8, shared) . B (s8, shared)^T, K 32.
-__device__ __forceinline__ void mma_i8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc) {
+// D (s32, tensor memory) = A (s8, tensor memory) . B (s8, shared)^T, K 32.
+__device__ __forceinline__ void mma_i8(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, 0, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc)
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc)
       : "memory");
+}
+
+// Eight 32-bit columns of this warp's 32 tensor-memory lanes.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -353,7 +364,6 @@ __global__ void __launch_bounds__(NT, 1) w4i_gemv_kernel(const __grid_constant__
   const int c1 = static_cast<int>(p.first[blockIdx.x + 1]);
 
   uint8_t* wst = smem + OFF_W;
-  uint8_t* asl = smem + OFF_A;
   uint8_t* ssl = smem + OFF_S;
   uint8_t* bsl = smem + OFF_B;
   uint8_t* zrow = smem + OFF_Z;
@@ -488,12 +498,12 @@ __global__ void __launch_bounds__(NT, 1) w4i_gemv_kernel(const __grid_constant__
         // (SBO = the distance from the digits to it, so it shrinks by 256
         // bytes with each K-step while the start grows by 256)
         const uint32_t bstart = smem_u32(bsl + ((tile - 1) & 1) * BSLOT) + static_cast<uint32_t>(GB * w.g * 256);
-        const uint64_t ad = sdesc(smem_u32(asl + a * ASLOT), 256u);
+        const uint32_t at = tmem + TA0 + static_cast<uint32_t>(a * GB * 8);
         const uint64_t bd = sdesc(bstart, smem_u32(zrow) - bstart);
         constexpr uint64_t BSTEP = static_cast<uint64_t>(256u >> 4) - (static_cast<uint64_t>(256u >> 4) << 32);
         const uint32_t dt = tmem + static_cast<uint32_t>(sl * GB * 16);
         for (int q = 0; q < nbg; ++q)
-          mma_i8(dt + 16 * q, ad + static_cast<uint64_t>((q * AB) >> 4), bd + static_cast<uint64_t>(q) * BSTEP, IDESC);
+          mma_i8(dt + 16 * q, at + 8 * q, bd + static_cast<uint64_t>(q) * BSTEP, IDESC);
         mma_commit(&afree[a]);
         mma_commit(&dready[sl]);
         lastG = w.G;
@@ -623,9 +633,11 @@ __global__ void __launch_bounds__(NT, 1) w4i_gemv_kernel(const __grid_constant__
     }
   } else if (warp >= 4 && warp != 8 && warp != 9 && warp != 10 && warp != 11) {
     // ------------------------------------------------------------ decode (warps 4-7 and 12-15)
-    // two teams of four; team t takes the groups G with G % 2 == t, warp j
-    // of the team block j of the group
+    // two teams of four; team t takes the groups G with G % 2 == t; warp j
+    // of the team decodes columns 32 j .. 32 j + 31 (its tensor-memory lanes)
+    // of every block of the group and copies block j's scales
     const int team = warp >= 12 ? 1 : 0, j = warp & 3;
+    const uint32_t lanes = static_cast<uint32_t>(32 * j) << 16;
     const long long budget = static_cast<long long>(p.timeout_ns) * 2;  // clocks, at most 2 per ns
     if (any) {
       GroupWalk w{c0, c1, 0, 0, 0, 0, 0, 0};
@@ -640,33 +652,36 @@ __global__ void __launch_bounds__(NT, 1) w4i_gemv_kernel(const __grid_constant__
           okw = poll_wait(&sfree[sl], static_cast<uint32_t>(w.G / NS - 1) & 1u, budget, abort_flag, p.err, 10);
         if (!__all_sync(0xffffffffu, okw)) break;
         const int nbg = min(GB, w.nb - GB * w.g);
-        if (j < nbg) {
-          const uint8_t* src = wst + s * GBYTES + j * BLK;
-          uint8_t* dst = asl + a * ASLOT + j * AB;
+        const uint8_t* stg = wst + s * GBYTES;
+        const int c = 32 * j + lane;  // column of the tile = tensor-memory lane
+        // A column 8 b + i of lane c: code bytes 4 i .. 4 i + 3 of block b
+        const uint32_t at = tmem + lanes + TA0 + static_cast<uint32_t>(a * GB * 8);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = lane + 32 * i;
-            const uint4 nib = *reinterpret_cast<const uint4*>(src + c * 16);
-            uint4 h0, h1;
-            h0.x = nib.x & 0x0F0F0F0Fu;
-            h0.y = (nib.x >> 4) & 0x0F0F0F0Fu;
-            h0.z = nib.y & 0x0F0F0F0Fu;
-            h0.w = (nib.y >> 4) & 0x0F0F0F0Fu;
-            h1.x = nib.z & 0x0F0F0F0Fu;
-            h1.y = (nib.z >> 4) & 0x0F0F0F0Fu;
-            h1.z = nib.w & 0x0F0F0F0Fu;
-            h1.w = (nib.w >> 4) & 0x0F0F0F0Fu;
-            uint8_t* ap = dst + (c >> 3) * 256 + (c & 7) * 16;
-            *reinterpret_cast<uint4*>(ap) = h0;
-            *reinterpret_cast<uint4*>(ap + 128) = h1;
+        for (int b = 0; b < GB; ++b) {
+          if (b < nbg) {
+            const uint4 nib = *reinterpret_cast<const uint4*>(stg + b * BLK + c * 16);
+            uint32_t v[8];
+            v[0] = nib.x & 0x0F0F0F0Fu;
+            v[1] = (nib.x >> 4) & 0x0F0F0F0Fu;
+            v[2] = nib.y & 0x0F0F0F0Fu;
+            v[3] = (nib.y >> 4) & 0x0F0F0F0Fu;
+            v[4] = nib.z & 0x0F0F0F0Fu;
+            v[5] = (nib.z >> 4) & 0x0F0F0F0Fu;
+            v[6] = nib.w & 0x0F0F0F0Fu;
+            v[7] = (nib.w >> 4) & 0x0F0F0F0Fu;
+            tmem_st8(at + 8 * b, v);
           }
-          // the block's scales (512 bytes) and zero points (64 bytes)
+        }
+        if (j < nbg) {
+          // block j's scales (512 bytes) and zero points (64 bytes)
+          const uint8_t* src = stg + j * BLK;
           uint8_t* sdst = ssl + sl * SSLOT + j * SZ;
           *reinterpret_cast<uint4*>(sdst + 16 * lane) = *reinterpret_cast<const uint4*>(src + 2048 + 16 * lane);
           if (lane < 4)
             *reinterpret_cast<uint4*>(sdst + 512 + 16 * lane) = *reinterpret_cast<const uint4*>(src + 2560 + 16 * lane);
         }
-        fence_async_smem();  // A is read by the tensor core
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();  // A is read by the tensor core
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&aready[a]);
