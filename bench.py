@@ -266,6 +266,15 @@ class Workload:
         if st != 0:
             raise RuntimeError(f"i8r_head_logits failed: {st} {self.lib.w4_last_error()}")
 
+    def step_fused(self, r: int, stream_handle: int):
+        """The whole decode step in one launch: the 48 repacked weights and
+        the head in its streaming layout, streamed by the same CTAs."""
+        rdescs, tr = self.copies[r][4], self.copies[r][6]
+        st = self.lib.w4r_decode_step(rdescs, len(rdescs), self.h.data_ptr(), tr.data_ptr(), HEAD_K, HEAD_V,
+                                      self.logits.data_ptr(), stream_handle)
+        if st != 0:
+            raise RuntimeError(f"w4r_decode_step failed: {st} {self.lib.w4_last_error()}")
+
     def head_tile(self, r: int, stream_handle: int):
         """The int8 head on the tensor cores (tile layout, integer MMAs)."""
         tt = self.copies[r][7]
@@ -298,16 +307,18 @@ def run_ours(args, world, rank, local):
     sh = int(stream.cuda_stream)
     warm = max(3, args.warmup)
     for i in range(warm):
+        wl.step_fused(i % R, sh)
         wl.body(i % R, sh)
         wl.head(i % R, sh)
     torch.cuda.synchronize()
 
     # ---- device-resident timing (value, roofline). Launch-bound work (a step
-    # is two launches of a few tens of microseconds), so the K timed steps are
+    # is one launch of about twenty microseconds), so the K timed steps are
     # captured in one CUDA graph and replayed on the stream the timing events
-    # are recorded on; an untimed replay uploads each graph first. The body and
-    # head kernels are also timed alone, K back-to-back launches each, for
-    # their average launch duration (the roofline).
+    # are recorded on; an untimed replay uploads each graph first. The step
+    # is one launch (w4r_decode_step), so its average launch duration is the
+    # step time; the same step as two launches (body, then head) and the body
+    # and head kernels alone are timed the same way for comparison.
     K = args.steps
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -346,7 +357,8 @@ def run_ours(args, world, rank, local):
         one = max_over_ranks(timed(g), world)
         return max(1, int(round(seconds * 1e3 / max(one, 1e-3))))
 
-    g_step = capture([wl.body, wl.head])
+    g_step = capture([wl.step_fused])
+    g_two = capture([wl.body, wl.head])
     g_body = capture([wl.body])
     g_head = capture([wl.head])
     g_page = capture([wl.body_page_format])
@@ -354,6 +366,7 @@ def run_ours(args, world, rank, local):
     g_htile = capture([wl.head_tile])
     g_step_t = capture([wl.body, wl.head_tile])
     n_step = reps_for(g_step, args.seconds)
+    n_two = reps_for(g_two, args.seconds / 2)
     n_body = reps_for(g_body, args.seconds / 2)
     n_head = reps_for(g_head, args.seconds / 2)
     n_page = reps_for(g_page, args.seconds / 4)
@@ -364,6 +377,7 @@ def run_ours(args, world, rank, local):
     sampler.start()
     time.sleep(0.2)
     total_ms = max_over_ranks(timed(g_step, n_step), world)
+    two_avg = timed(g_two, n_two) / (K * n_two)
     body_avg = timed(g_body, n_body) / (K * n_body)
     head_avg = timed(g_head, n_head) / (K * n_head)
     page_avg = timed(g_page, n_page) / (K * n_page)
@@ -373,13 +387,14 @@ def run_ours(args, world, rank, local):
     clocks = sampler.stop()
     steps_timed = K * n_step
     ms_step = total_ms / steps_timed
-    del g_step, g_body, g_head, g_page, g_hpage, g_htile, g_step_t
+    del g_step, g_two, g_body, g_head, g_page, g_hpage, g_htile, g_step_t
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(wl, args, world, R)
 
     peaks = measured_peaks()
-    achieved = body_bytes() / (body_avg * 1e-3) / 1e9
+    achieved = step_bytes / (ms_step * 1e-3) / 1e9  # the step's one launch
+    body_achieved = body_bytes() / (body_avg * 1e-3) / 1e9
     n = world
     value = whole_job_gbs(step_bytes, n, ms_step)
     line = {
@@ -406,15 +421,21 @@ def run_ours(args, world, rank, local):
             "parallelism": f"replicas x{n}" if n > 1 else "1 GPU",
             "l2": f"rotating {R} weight copies ({R * step_bytes / 1e6:.0f} MB, > 3x L2): every step L2-cold",
             "seed": synth.BASE_SEED,
-            "body_path": "48 weights in the streaming layout (repacked once at load, same bytes), "
-                         "w4r_matmul_grouped; head in its streaming layout, i8r_head_logits",
+            "body_path": "one launch per step (w4r_decode_step): the 48 weights in the streaming layout "
+                         "(repacked once at load, same bytes) and the head in its streaming layout, streamed by "
+                         "the same persistent CTAs",
             "timing": "a CUDA graph of K steps replayed back to back for about --seconds, CUDA events on the "
-                      "replay stream; body_only/head_only (roofline): K launches of that kernel alone per graph, "
-                      "replayed the same way",
+                      "replay stream; step_two_launches, body_only, head_only: K steps (launches) of that "
+                      "form per graph, replayed the same way",
         },
         "tokens_per_s": round(n * 1e3 / ms_step, 1),
-        "body_only": {"ms": round(body_avg, 5), "GB_per_s": round(achieved, 1),
-                      "tokens_per_s": round(1e3 / body_avg, 1), "launches_timed": K * n_body},
+        "step_two_launches": {"ms": round(two_avg, 5),
+                              "GB_per_s": round(step_bytes / (two_avg * 1e-3) / 1e9, 1),
+                              "kernels": "w4r_gemv_m1_kernel<false> (48 weights), then i8r_head_kernel"},
+        "body_only": {"ms": round(body_avg, 5), "GB_per_s": round(body_achieved, 1),
+                      "frac_of_hbm": round(body_achieved / peaks["hbm_gbs"], 4),
+                      "tokens_per_s": round(1e3 / body_avg, 1), "launches_timed": K * n_body,
+                      "traffic": profiled_traffic("w4r_gemv_gpt2_m1.md")},
         "body_page_format": {"ms": round(page_avg, 5),
                              "GB_per_s": round(body_bytes() / (page_avg * 1e-3) / 1e9, 1),
                              "kernel": "w4_gemv_kernel<1> (split-K GEMV on the page-format buffers)"},
@@ -432,19 +453,20 @@ def run_ours(args, world, rank, local):
                              "kernel": "i8_rows_kernel<1> (page-format table)"},
         "frac_of_hbm_step": round(value / n / peaks["hbm_gbs"], 4),
         "roofline": {
-            "kernel": "w4r_gemv_m1_kernel (48 repacked weights, one grouped launch)",
+            "kernel": "w4r_gemv_m1_kernel<true> (the decode step: 48 repacked weights and the head, one launch)",
             "bound": "hbm",
             "achieved": round(achieved, 1),
+            "algorithmic_bytes_per_launch": step_bytes,
             "peak": peaks["hbm_gbs"],
             "peak_source": f"{peaks['_source']} hbm_gbs (copy, burst)",
             "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": profiled_traffic("w4r_gemv_gpt2_m1.md"),
-            "traffic_source": "profiles/w4r_gemv_gpt2_m1.md (ncu dram__bytes_read.sum + dram__bytes_write.sum, "
+            "traffic": profiled_traffic("w4r_step_gpt2_m1.md"),
+            "traffic_source": "profiles/w4r_step_gpt2_m1.md (ncu dram__bytes_read.sum + dram__bytes_write.sum, "
                               "one launch; null when the kernel source changed since)",
         },
         "e2e": e2e,
-        "gpu_launches": 2 * steps_timed,  # body + head per step in the timed replays
+        "gpu_launches": steps_timed,  # one launch per step in the timed replays
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -456,9 +478,8 @@ def run_ours(args, world, rank, local):
 
 def run_e2e(wl, args, world, R):
     """Same step through the public binding with host buffers: per step, copy
-    the step's inputs from pinned host memory, run body + head, read every
-    output back to pinned host memory (the body's outputs while the head
-    runs)."""
+    the step's inputs from pinned host memory, run the step (one launch), read
+    every output back to pinned host memory."""
     import torch
     stream = torch.cuda.current_stream()
     sh = int(stream.cuda_stream)
@@ -467,22 +488,10 @@ def run_e2e(wl, args, world, R):
     h2d = inh.numel() * 4
     d2h = outh.numel() * 4
 
-    # the 48 outputs go back on a second stream while the head runs; the
-    # logits follow the head on the main stream
-    side = torch.cuda.Stream()
-    body_done = torch.cuda.Event()
-    ny = wl.out_dev.numel() - wl.logits.numel()
-
     def step(r):
         wl.in_dev.copy_(inh, non_blocking=True)
-        wl.body(r, sh)
-        body_done.record(stream)
-        wl.head(r, sh)
-        side.wait_event(body_done)
-        with torch.cuda.stream(side):
-            outh[:ny].copy_(wl.out_dev[:ny], non_blocking=True)
-        outh[ny:].copy_(wl.out_dev[ny:], non_blocking=True)
-        stream.wait_stream(side)  # the step ends when both copies have
+        wl.step_fused(r, sh)
+        outh.copy_(wl.out_dev, non_blocking=True)
 
     for i in range(3):
         step(i % R)
@@ -967,8 +976,9 @@ def run_reference(args, world, rank):
 
 def profile_case(name: str, calls: int) -> None:
     """Run one workload's kernels `calls` times (no timing, no output but one
-    line) so that a profiler can capture them: "body" (the 48 GPT-2 weights
-    in the streaming layout, M = 1), "head" (the int8 head, streaming
+    line) so that a profiler can capture them: "step" (the decode step in one
+    launch: the 48 GPT-2 weights and the head, streaming layouts, M = 1),
+    "body" (the 48 GPT-2 weights in the streaming layout, M = 1), "head" (the int8 head, streaming
     layout, M = 1), "head-tile" / "head-tile-m8" (the int8 head in the tile
     layout, tensor cores, M = 1 / 8), "prefill-gpt2" (the 48 weights in the tile layout at
     M = 58), "prefill-3p8b" (one 3.8B-shaped layer, 4 weights in the tile
@@ -978,19 +988,27 @@ def profile_case(name: str, calls: int) -> None:
     dev = torch.device("cuda", 0)
     lib = w4.lib()
     hs = int(torch.cuda.current_stream().cuda_stream)
-    if name in ("body", "prefill-gpt2", "prefill-3p8b"):
+    if name in ("body", "step", "prefill-gpt2", "prefill-3p8b"):
         shapes = synth.gpt2_stack_shapes() if name != "prefill-3p8b" else synth.dense38_stack_shapes()[:4]
-        M = {"body": 1, "prefill-gpt2": synth.GPT2_PROMPT, "prefill-3p8b": 2048}[name]
+        M = {"body": 1, "step": 1, "prefill-gpt2": synth.GPT2_PROMPT, "prefill-3p8b": 2048}[name]
         items = []
         for i, (_, K, N) in enumerate(shapes):
             W = synth.w4_weight(K, N, i)
             qw, sc, zp = (torch.from_numpy(W[k]).to(dev) for k in ("qw", "scales", "zp"))
-            rep = w4.w4_repack if name == "body" else w4.w4t_repack
+            rep = w4.w4_repack if name in ("body", "step") else w4.w4t_repack
             items.append({"x": torch.from_numpy(synth.activations(M, K, i)).to(dev), "wr": rep(qw, sc, zp, K, N),
                           "y": torch.empty((M, N), device=dev), "K": K, "N": N})
         descs = w4.make_rdescs(items)
         if name == "body":
             run = lambda: _ok(lib.w4r_matmul_grouped(descs, len(descs), hs), lib, "w4r")
+        elif name == "step":
+            H = synth.i8_head(HEAD_K, HEAD_V)
+            tr = w4.i8_head_repack(torch.from_numpy(H["table"]).to(dev), torch.from_numpy(H["scales"]).to(dev),
+                                   HEAD_K, HEAD_V)
+            h = torch.from_numpy(synth.activations(1, HEAD_K, 999)).to(dev)
+            lg = torch.empty((1, HEAD_V), device=dev)
+            run = lambda: _ok(lib.w4r_decode_step(descs, len(descs), h.data_ptr(), tr.data_ptr(), HEAD_K, HEAD_V,
+                                                  lg.data_ptr(), hs), lib, "w4r_decode_step")
         else:
             scratch = torch.empty(max(w4.w4t_workspace_size(descs), 16), dtype=torch.uint8, device=dev)
             run = lambda: _ok(lib.w4t_matmul_grouped(descs, len(descs), scratch.data_ptr(), scratch.numel(), hs), lib,
@@ -1032,7 +1050,7 @@ def main():
                     help="device seconds of the timed step replays (the body and head alone get half each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config measurements (configs 0, 2, 3, 4)")
-    ap.add_argument("--profile-case", choices=["body", "head", "head-tile", "head-tile-m8", "prefill-gpt2", "prefill-3p8b"],
+    ap.add_argument("--profile-case", choices=["step", "body", "head", "head-tile", "head-tile-m8", "prefill-gpt2", "prefill-3p8b"],
                     default=None,
                     help="only run one workload's kernels a few times, for a profiler (see profiles/)")
     ap.add_argument("--calls", type=int, default=4, help="calls of --profile-case")

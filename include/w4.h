@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define W4_ABI_VERSION 5
+#define W4_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define W4_API __attribute__((visibility("default")))
@@ -416,6 +416,28 @@ W4_API w4_status i8r_head_logits(const float* h, const void* tr, int64_t K, int6
  * 8 bytes of device memory (8-byte aligned) that the call clears and uses. */
 W4_API w4_status i8r_head_argmax(const float* h, const void* tr, int64_t K, int64_t V, int32_t* token,
                                  float* best_logit, void* keys, void* stream);
+
+/* One decode step in one launch: the matmuls of `descs` (as
+ * w4r_matmul_grouped: repacked weights, M = 1) and the int8 head's logits
+ * (as i8r_head_logits: logits[v] = s_v * sum_k h_k T[k, v] on the head in its
+ * streaming layout), streamed by the same persistent CTAs, each of which takes
+ * an equal share of the body's column groups and of the head's, so that the
+ * step pays one launch's start and tail ("ONNX export, quantization and the
+ * browser runtime", section "Quantization (train/quantize.py)", steps 2 to
+ * 4). Every output is bit-identical to the two separate calls.
+ * - descs / count: as for w4r_matmul_grouped (a HOST array, read during the
+ *   call only; count may be 0).
+ * - h, tr, K, V, logits: as for i8r_head_logits. h is read when the launch
+ *   starts, so it must not overlap any y of `descs` (W4_ERR_VALUE): within a
+ *   step the head's input is not one of the body's outputs.
+ * - A step that one launch cannot hold (more than 64 weights, K of the head
+ *   above 2048, or more x than a CTA stages) runs as the body's launches
+ *   followed by the head's, with the same results.
+ * - The launch starts streaming while the previous work on the stream
+ *   finishes (programmatic dependent launch); x and h are read and y and the
+ *   logits written only after that work has completed. */
+W4_API w4_status w4r_decode_step(const w4r_desc* descs, int32_t count, const float* h, const void* tr, int64_t K,
+                                 int64_t V, float* logits, void* stream);
 
 /* The tile layout of the int8 head, read by the tensor-core head
  * (i8t_head_logits / i8t_head_argmax) for 1 to 8 last-position rows. The

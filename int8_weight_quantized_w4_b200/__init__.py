@@ -431,6 +431,19 @@ def i8r_head_logits(h, tr, K: int, V: int, logits=None, stream=None):
     return logits
 
 
+def w4r_decode_step(items: Sequence[dict] | None, h, tr, K: int, V: int, logits=None, descs=None, stream=None):
+    """One decode step in one launch: the matmuls of `items` (or a prepared
+    w4r_desc array) and the head's logits [1, V] of h on the repacked head."""
+    torch = _torch()
+    if descs is None:
+        descs = make_rdescs(items or [])
+    if logits is None:
+        logits = torch.empty((1, V), dtype=torch.float32, device=h.device)
+    _check(lib().w4r_decode_step(descs, len(descs), _ptr(h), _ptr(tr), K, V, _ptr(logits), _stream_handle(stream)),
+           "w4r_decode_step")
+    return logits
+
+
 def i8r_head_argmax(h, tr, K: int, V: int, stream=None):
     """(token int32 [1], best logit fp32 [1]) of one row h on a repacked head."""
     torch = _torch()

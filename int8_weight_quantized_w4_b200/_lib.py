@@ -27,7 +27,7 @@ W4_OK, W4_ERR_NULL, W4_ERR_SHAPE, W4_ERR_ALIGN, W4_ERR_DEVICE, W4_ERR_CUDA, W4_E
     W4_ERR_VALUE = range(9)
 PATHS = {"auto": 0, "gemv": 1, "generic": 2, "tc": 3}
 ACTS = {"none": 0, "gelu_tanh": 1, "gelu_erf": 2}
-ABI_VERSION = 5
+ABI_VERSION = 6
 GROUP_MAX = 48
 
 
@@ -103,6 +103,8 @@ SIGNATURES = {
     "i8_head_repack_restore": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p,
                                          C.c_void_p]),
     "i8r_head_logits": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),
+    "w4r_decode_step": (C.c_int, [C.POINTER(W4RDesc), C.c_int32, C.c_void_p, C.c_void_p, C.c_int64, C.c_int64,
+                                  C.c_void_p, C.c_void_p]),
     "i8t_head_repacked_bytes": (C.c_size_t, [C.c_int64, C.c_int64]),
     "i8t_head_repack": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),
     "i8t_head_repack_restore": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p,

@@ -48,42 +48,13 @@ namespace {
 
 using namespace w4dev;
 
-constexpr int HROUND = 4096;            // table bytes of a round
+constexpr int HROUND = w4host::kStreamHeadRound;  // table bytes of a round
 constexpr int HSTAGE = HROUND + 1024;   // a round plus up to 32 * 8 scales
 constexpr int HW = 12;                  // warps per CTA
 constexpr int HST = 3;                  // stages per warp
-constexpr int HKCAP = 8192;             // rows of h a CTA can hold
+constexpr int HKCAP = w4host::kStreamHeadKCap;    // rows of h a CTA can hold
 constexpr int HSTAGE_SMEM = HW * HST * HSTAGE;
 constexpr int HSMEM_BYTES = HSTAGE_SMEM + HKCAP * 4 + HW * HST * 8 + HW * 4;
-
-struct HeadGeom {
-  int32_t nb, gsl, A, ngroups;
-  int64_t group_bytes;
-  int64_t bytes;
-};
-
-int gcd32(int a) {
-  int b = 32;
-  while (b != 0) {
-    const int t = a % b;
-    a = b;
-    b = t;
-  }
-  return a;
-}
-
-bool head_geom(int64_t K, int64_t V, HeadGeom* g) {
-  if (K <= 0 || V <= 0 || K % 16 != 0 || K > HKCAP || V > (int64_t(1) << 30)) return false;
-  g->nb = static_cast<int32_t>(K / 16);
-  const int gs = 32 / gcd32(g->nb);
-  g->gsl = __builtin_ctz(gs);
-  g->A = g->nb / gcd32(g->nb);
-  const int64_t strips = (V + 7) / 8;
-  g->ngroups = static_cast<int32_t>((strips + gs - 1) / gs);
-  g->group_bytes = static_cast<int64_t>(g->A) * HROUND + 32 * gs;
-  g->bytes = g->ngroups * g->group_bytes;
-  return true;
-}
 
 struct HParams {
   const uint8_t* tr;
@@ -103,45 +74,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
-// Byte j of a biased word in the mantissa of 2^23: [byte j, 0, 0, 0x4B].
-template <int J>
-__device__ __forceinline__ float byte_float(uint32_t w, uint32_t magic) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(w), "r"(magic), "n"(0x7540 | J));
-  return __uint_as_float(r);
-}
-
-// One 16-row x 8-column atom of this lane into P[0..7] (two running sums per
-// column, rows 2c and 2c+1). hb: h of the atom's block, row pair c at
-// hb + c * hq floats.
-__device__ __forceinline__ void atom_i8(const uint8_t* st, int lane, const float* hb, int hq, uint32_t magic,
-                                        float2 nbias, float2 (&P)[8]) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint4 wv = *reinterpret_cast<const uint4*>(st + c * 512 + lane * 16);
-    const float2 hv = *reinterpret_cast<const float2*>(hb + c * hq);
-    // wv.x: row 2c cols 0-3, wv.y: row 2c cols 4-7, wv.z / wv.w: row 2c+1
-    P[0] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<0>(wv.x, magic), byte_float<0>(wv.z, magic)), nbias), P[0]);
-    P[1] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<1>(wv.x, magic), byte_float<1>(wv.z, magic)), nbias), P[1]);
-    P[2] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<2>(wv.x, magic), byte_float<2>(wv.z, magic)), nbias), P[2]);
-    P[3] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<3>(wv.x, magic), byte_float<3>(wv.z, magic)), nbias), P[3]);
-    P[4] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<0>(wv.y, magic), byte_float<0>(wv.w, magic)), nbias), P[4]);
-    P[5] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<1>(wv.y, magic), byte_float<1>(wv.w, magic)), nbias), P[5]);
-    P[6] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<2>(wv.y, magic), byte_float<2>(wv.w, magic)), nbias), P[6]);
-    P[7] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<3>(wv.y, magic), byte_float<3>(wv.w, magic)), nbias), P[7]);
-  }
-}
-
-// Order-preserving 64-bit key of (logit, token): logit bits made monotonic
-// (-0 taken as +0) above the complement of the token id, so the maximum key
-// is the largest logit and, among equal logits, the lowest id.
-__device__ __forceinline__ unsigned long long head_key(float logit, uint32_t token) {
-  uint32_t b = __float_as_uint(logit);
-  if (b == 0x80000000u) b = 0u;
-  const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-  return (static_cast<unsigned long long>(o) << 32) | static_cast<unsigned long long>(0xFFFFFFFFu - token);
-}
 
 __global__ void __launch_bounds__(HW * 32, 1) i8r_head_kernel(const __grid_constant__ HParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -294,7 +226,7 @@ __global__ void __launch_bounds__(HW * 32, 1) i8r_head_kernel(const __grid_const
 
 // Source of byte-word o of the repacked head: kind 0 a table word (4
 // columns of one row), 1 a scale; fills *row / *col (first column).
-__device__ __forceinline__ int head_source(int64_t o, const HeadGeom& g, int* row, int64_t* col) {
+__device__ __forceinline__ int head_source(int64_t o, const w4host::StreamHeadGeom& g, int* row, int64_t* col) {
   const int64_t gw = g.group_bytes / 4;
   const int64_t G = o / gw;
   const int w = static_cast<int>(o - G * gw);
@@ -314,7 +246,7 @@ __device__ __forceinline__ int head_source(int64_t o, const HeadGeom& g, int* ro
 }
 
 __global__ void i8r_repack_kernel(const int8_t* __restrict__ table, int64_t ldt, const float* __restrict__ scales,
-                                  int64_t V, HeadGeom g, uint32_t* __restrict__ out) {
+                                  int64_t V, w4host::StreamHeadGeom g, uint32_t* __restrict__ out) {
   const int64_t words = g.bytes / 4;
   for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < words;
        o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -335,7 +267,7 @@ __global__ void i8r_repack_kernel(const int8_t* __restrict__ table, int64_t ldt,
   }
 }
 
-__global__ void i8r_restore_kernel(const uint32_t* __restrict__ in, int64_t V, HeadGeom g, int8_t* __restrict__ table,
+__global__ void i8r_restore_kernel(const uint32_t* __restrict__ in, int64_t V, w4host::StreamHeadGeom g, int8_t* __restrict__ table,
                                    int64_t ldt, float* __restrict__ scales) {
   const int64_t words = g.bytes / 4;
   for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < words;
@@ -359,8 +291,8 @@ bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t
 w4_status launch_i8r(const float* h, const void* tr, int64_t K, int64_t V, float* logits, unsigned long long* keys,
                      cudaStream_t st, const w4host::DeviceInfo& di) {
   using namespace w4host;
-  HeadGeom g;
-  head_geom(K, V, &g);
+  w4host::StreamHeadGeom g;
+  w4host::stream_head_geom(K, V, &g);
   HParams prm = {};
   prm.tr = static_cast<const uint8_t*>(tr);
   prm.h = h;
@@ -396,8 +328,8 @@ w4_status launch_i8r(const float* h, const void* tr, int64_t K, int64_t V, float
 
 w4_status check_head_args(const float* h, const void* tr, int64_t K, int64_t V) {
   using namespace w4host;
-  HeadGeom g;
-  if (!head_geom(K, V, &g))
+  w4host::StreamHeadGeom g;
+  if (!w4host::stream_head_geom(K, V, &g))
     return fail(W4_ERR_SHAPE, "the streaming head takes K %% 16 == 0, 0 < K <= %d and 0 < V <= 2^30 (K=%lld V=%lld)",
                 HKCAP, static_cast<long long>(K), static_cast<long long>(V));
   if (h == nullptr || tr == nullptr) return fail(W4_ERR_NULL, "h and the repacked table must not be NULL");
@@ -408,18 +340,54 @@ w4_status check_head_args(const float* h, const void* tr, int64_t K, int64_t V) 
 
 }  // namespace
 
+namespace w4host {
+
+namespace {
+int gcd32(int a) {
+  int b = 32;
+  while (b != 0) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+}  // namespace
+
+bool stream_head_geom(int64_t K, int64_t V, StreamHeadGeom* g) {
+  if (K <= 0 || V <= 0 || K % 16 != 0 || K > kStreamHeadKCap || V > (int64_t(1) << 30)) return false;
+  g->nb = static_cast<int32_t>(K / 16);
+  const int gs = 32 / gcd32(g->nb);
+  g->gsl = __builtin_ctz(gs);
+  g->A = g->nb / gcd32(g->nb);
+  const int64_t strips = (V + 7) / 8;
+  g->ngroups = static_cast<int32_t>((strips + gs - 1) / gs);
+  g->group_bytes = static_cast<int64_t>(g->A) * kStreamHeadRound + 32 * gs;
+  g->bytes = g->ngroups * g->group_bytes;
+  return true;
+}
+
+w4_status check_stream_head(const float* h, const void* tr, int64_t K, int64_t V) { return check_head_args(h, tr, K, V); }
+
+w4_status launch_stream_head(const float* h, const void* tr, int64_t K, int64_t V, float* logits, cudaStream_t st,
+                             const DeviceInfo& di) {
+  return launch_i8r(h, tr, K, V, logits, nullptr, st, di);
+}
+
+}  // namespace w4host
+
 extern "C" {
 
 size_t i8_head_repacked_bytes(int64_t K, int64_t V) {
-  HeadGeom g;
-  return head_geom(K, V, &g) ? static_cast<size_t>(g.bytes) : 0;
+  w4host::StreamHeadGeom g;
+  return w4host::stream_head_geom(K, V, &g) ? static_cast<size_t>(g.bytes) : 0;
 }
 
 w4_status i8_head_repack(const int8_t* table, int64_t ldt, const float* scales, int64_t K, int64_t V, void* tr,
                          void* stream) {
   using namespace w4host;
-  HeadGeom g;
-  if (!head_geom(K, V, &g))
+  w4host::StreamHeadGeom g;
+  if (!w4host::stream_head_geom(K, V, &g))
     return fail(W4_ERR_SHAPE, "the streaming head takes K %% 16 == 0, 0 < K <= %d and 0 < V <= 2^30", HKCAP);
   if (ldt < V) return fail(W4_ERR_SHAPE, "ldt < V");
   if (table == nullptr || scales == nullptr || tr == nullptr) return fail(W4_ERR_NULL, "NULL buffer");
@@ -437,8 +405,8 @@ w4_status i8_head_repack(const int8_t* table, int64_t ldt, const float* scales, 
 w4_status i8_head_repack_restore(const void* tr, int64_t K, int64_t V, int8_t* table, int64_t ldt, float* scales,
                                  void* stream) {
   using namespace w4host;
-  HeadGeom g;
-  if (!head_geom(K, V, &g))
+  w4host::StreamHeadGeom g;
+  if (!w4host::stream_head_geom(K, V, &g))
     return fail(W4_ERR_SHAPE, "the streaming head takes K %% 16 == 0, 0 < K <= %d and 0 < V <= 2^30", HKCAP);
   if (ldt < V) return fail(W4_ERR_SHAPE, "ldt < V");
   if (table == nullptr || scales == nullptr || tr == nullptr) return fail(W4_ERR_NULL, "NULL buffer");

@@ -230,4 +230,46 @@ __device__ __forceinline__ float epi_apply(float v, const Epi& e, int64_t m, int
   return v;
 }
 
+// ---- the int8 head's streaming-layout atom (shared by the head kernel and
+// the fused decode step)
+
+// Byte j of a biased word in the mantissa of 2^23: [byte j, 0, 0, 0x4B].
+template <int J>
+__device__ __forceinline__ float byte_float(uint32_t w, uint32_t magic) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(w), "r"(magic), "n"(0x7540 | J));
+  return __uint_as_float(r);
+}
+
+// One 16-row x 8-column atom of this lane into P[0..7] (two running sums per
+// column, rows 2c and 2c+1). hb: h of the atom's block, row pair c at
+// hb + c * hq floats.
+__device__ __forceinline__ void atom_i8(const uint8_t* st, int lane, const float* hb, int hq, uint32_t magic,
+                                        float2 nbias, float2 (&P)[8]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 wv = *reinterpret_cast<const uint4*>(st + c * 512 + lane * 16);
+    const float2 hv = *reinterpret_cast<const float2*>(hb + c * hq);
+    // wv.x: row 2c cols 0-3, wv.y: row 2c cols 4-7, wv.z / wv.w: row 2c+1
+    P[0] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<0>(wv.x, magic), byte_float<0>(wv.z, magic)), nbias), P[0]);
+    P[1] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<1>(wv.x, magic), byte_float<1>(wv.z, magic)), nbias), P[1]);
+    P[2] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<2>(wv.x, magic), byte_float<2>(wv.z, magic)), nbias), P[2]);
+    P[3] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<3>(wv.x, magic), byte_float<3>(wv.z, magic)), nbias), P[3]);
+    P[4] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<0>(wv.y, magic), byte_float<0>(wv.w, magic)), nbias), P[4]);
+    P[5] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<1>(wv.y, magic), byte_float<1>(wv.w, magic)), nbias), P[5]);
+    P[6] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<2>(wv.y, magic), byte_float<2>(wv.w, magic)), nbias), P[6]);
+    P[7] = __ffma2_rn(hv, __fadd2_rn(make_float2(byte_float<3>(wv.y, magic), byte_float<3>(wv.w, magic)), nbias), P[7]);
+  }
+}
+
+// Order-preserving 64-bit key of (logit, token): logit bits made monotonic
+// (-0 taken as +0) above the complement of the token id, so the maximum key
+// is the largest logit and, among equal logits, the lowest id.
+__device__ __forceinline__ unsigned long long head_key(float logit, uint32_t token) {
+  uint32_t b = __float_as_uint(logit);
+  if (b == 0x80000000u) b = 0u;
+  const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return (static_cast<unsigned long long>(o) << 32) | static_cast<unsigned long long>(0xFFFFFFFFu - token);
+}
+
 }  // namespace w4dev

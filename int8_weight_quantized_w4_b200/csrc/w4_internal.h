@@ -76,6 +76,19 @@ w4_status launch_argmax_rows(const float* logits, int64_t ldl, int64_t M, int64_
 w4_status launch_argmax_finish(const unsigned long long* keys, int64_t M, int32_t* tokens, float* best,
                                cudaStream_t st);
 
+// ---- the head's streaming layout (i8r.cu), also read by the fused decode step
+constexpr int kStreamHeadRound = 4096;  // table bytes of a round
+constexpr int kStreamHeadKCap = 8192;   // rows of h the head kernel holds
+struct StreamHeadGeom {
+  int32_t nb, gsl, A, ngroups;  // 16-row blocks, log2 strips per group, rounds per group, groups
+  int64_t group_bytes;          // A rounds of table bytes, then 8 * 2^gsl scales
+  int64_t bytes;
+};
+bool stream_head_geom(int64_t K, int64_t V, StreamHeadGeom* g);
+w4_status check_stream_head(const float* h, const void* tr, int64_t K, int64_t V);
+w4_status launch_stream_head(const float* h, const void* tr, int64_t K, int64_t V, float* logits, cudaStream_t st,
+                             const DeviceInfo& di);
+
 // ---- diagnostics
 w4_status launch_debug_wait(uint64_t timeout_ns, cudaStream_t st, const DeviceInfo& di);
 

@@ -82,6 +82,12 @@ constexpr int RCAP = 64;                      // matrices per launch
 constexpr int XCAP = 8192;                    // floats of x a CTA can hold
 constexpr int STAGE_SMEM = PW * PST * ROUND_BYTES;
 constexpr int SMEM_BYTES = STAGE_SMEM + XCAP * 4 + PW * PST * 8 + PW * 4;
+// the fused decode step: the head's rounds share the stages, its h follows
+constexpr int HROUND = w4host::kStreamHeadRound;  // table bytes of a head round
+constexpr int HKS = 2048;                         // rows of the head's h a CTA of the step holds
+constexpr int SMEM_STEP = SMEM_BYTES + HKS * 4;
+static_assert(HROUND + 32 * 32 <= ROUND_BYTES, "a head round and its scales fit a stage");
+static_assert(SMEM_BYTES % 16 == 0 && SMEM_STEP <= 227 * 1024, "shared memory of one CTA");
 
 struct RMat {
   const uint8_t* wr;
@@ -98,10 +104,23 @@ struct RMat {
   int32_t gsl;      // log2(gs)
 };
 
+// The int8 head in its streaming layout, streamed by the same launch (the
+// fused decode step): groups of 8 * 2^gsl token columns, A rounds of table
+// bytes each, the group's scales after its last round.
+struct RHead {
+  const uint8_t* tr;
+  const float* h;
+  float* logits;
+  int64_t group_bytes;
+  int32_t K, V, gsl, A;
+};
+
 struct RParams {
   RMat m[RCAP];
   int32_t count;
-  int32_t T;  // groups of the launch
+  int32_t T;   // body groups of the launch
+  int32_t TH;  // head groups (the fused step; 0 otherwise)
+  RHead hd;
   ErrorWord* err;
   uint64_t timeout_ns;
 };
@@ -172,22 +191,37 @@ __device__ __forceinline__ void atom_m1(const uint8_t* st, int lane, const float
   for (int i = 0; i < 8; ++i) acc[i] = fmaf(P[i].x + P[i].y, sv[i] * inv_slot_scale(i & 3), acc[i]);
 }
 
-// The rounds one warp streams, in order: its groups lo + warp + PW t, each
-// of A rounds. Producer (lane 0) and consumers walk the same sequence.
+// The rounds one warp streams, in order: units u = warp + PW t of its CTA,
+// each a group of A rounds; unit u < nbc is body group lo + u, a later one
+// head group hlo + u - nbc. Producer (lane 0) and consumers walk the same
+// sequence.
 struct RoundWalk {
-  int t, r, ngw;  // group ordinal of this warp, round in it, groups of this warp
-  int g, A;       // matrix of the current group, its rounds per group
+  int t, r, ngw;  // unit ordinal of this warp, round in it, units of this warp
+  int g, A;       // matrix of the current body group, rounds of the current unit
   const uint8_t* base;
+  int rb, last;   // bytes between rounds; bytes of the unit's last round
 };
 
-__device__ __forceinline__ void walk_group(RoundWalk& w, const RParams& p, int lo, int warp) {
-  const int gg = lo + warp + PW * w.t;
+template <bool HEAD>
+__device__ __forceinline__ void walk_group(RoundWalk& w, const RParams& p, int lo, int nbc, int hlo, int warp) {
+  const int u = warp + PW * w.t;
+  if (HEAD && u >= nbc) {
+    w.A = p.hd.A;
+    w.base = p.hd.tr + static_cast<int64_t>(hlo + u - nbc) * p.hd.group_bytes;
+    w.rb = HROUND;
+    w.last = HROUND + (32 << p.hd.gsl);  // the group's scales ride on its last round
+    return;
+  }
+  const int gg = lo + u;
   while (w.g + 1 < p.count && p.m[w.g + 1].g0 <= gg) ++w.g;
   const RMat& m = p.m[w.g];
   w.A = ((m.K >> 5) << m.gsl) >> 5;
   w.base = m.wr + static_cast<int64_t>(gg - m.g0) * w.A * ROUND_BYTES;
+  w.rb = ROUND_BYTES;
+  w.last = ROUND_BYTES;
 }
 
+template <bool HEAD>
 __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_constant__ RParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
@@ -195,49 +229,66 @@ __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_co
   const int G = gridDim.x;
   const int lo = range_lo(blockIdx.x, p.T, G);
   const int hi = range_lo(blockIdx.x + 1, p.T, G);
-  const int ngw = hi - lo > warp ? (hi - lo - warp + PW - 1) / PW : 0;  // groups of this warp
+  const int nbc = hi - lo;  // body groups of this CTA
+  const int hlo = HEAD ? range_lo(blockIdx.x, p.TH, G) : 0;
+  const int nhc = HEAD ? range_lo(blockIdx.x + 1, p.TH, G) - hlo : 0;  // head groups of this CTA
+  const int units = nbc + nhc;
+  const int ngw = units > warp ? (units - warp + PW - 1) / PW : 0;  // units of this warp
 
   uint8_t* stg = smem + warp * (PST * ROUND_BYTES);
   float* xs = reinterpret_cast<float*>(smem + STAGE_SMEM);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + STAGE_SMEM + XCAP * 4) + warp * PST;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + STAGE_SMEM + XCAP * 4 + PW * PST * 8) + warp;
+  float* hs = reinterpret_cast<float*>(smem + SMEM_BYTES);  // the head's h (fused step only)
 
   // ---- x into L2 now: a cache hint only (the values are read after the
   // wait), so that the staging below does not queue behind weight bytes
   if (threadIdx.x == 0) {
-    const int g1 = hi > lo ? mat_of(p, hi - 1) : mat_of(p, lo);
-    for (int g = mat_of(p, lo); g <= g1; ++g)
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.m[g].x), "r"(p.m[g].K * 4) : "memory");
+    if (nbc > 0) {
+      const int g1 = mat_of(p, hi - 1);
+      for (int g = mat_of(p, lo); g <= g1; ++g)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.m[g].x), "r"(p.m[g].K * 4) : "memory");
+    }
+    if (HEAD && nhc > 0)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.hd.h), "r"(p.hd.K * 4) : "memory");
   }
   // ---- the first round of every warp before the wait: the weights do not
   // depend on the previous launch, so they stream while it finishes
-  const int gfirst = mat_of(p, lo);
-  RoundWalk iw{0, 0, ngw, gfirst, 0, nullptr};  // issue cursor, kept in step by every lane
+  const int gfirst = nbc > 0 ? mat_of(p, lo) : 0;
+  RoundWalk iw{0, 0, ngw, gfirst, 0, nullptr, 0, 0};  // issue cursor, kept in step by every lane
   int issued = 0;
+  // one bulk copy of the round under the cursor into stage `stage`; the
+  // cursor moves on (warp-uniform)
+  auto issue = [&](int stage) {
+    if (lane == 0) {
+      const uint32_t bytes = static_cast<uint32_t>(iw.r == iw.A - 1 ? iw.last : iw.rb);
+      mbar_arrive_expect_tx(&bar[stage], bytes);
+      bulk_g2s(stg + stage * ROUND_BYTES, iw.base + static_cast<int64_t>(iw.r) * iw.rb, bytes, &bar[stage]);
+    }
+    ++issued;
+    if (++iw.r == iw.A) {
+      iw.r = 0;
+      if (++iw.t < ngw) walk_group<HEAD>(iw, p, lo, nbc, hlo, warp);
+    }
+  };
   if (ngw > 0) {
-    walk_group(iw, p, lo, warp);
+    walk_group<HEAD>(iw, p, lo, nbc, hlo, warp);
     if (lane == 0) {
       for (int s = 0; s < PST; ++s) mbar_init(&bar[s], 1);
       *abort_flag = 0;
       fence_mbar_init();
-      mbar_arrive_expect_tx(&bar[0], ROUND_BYTES);
-      bulk_g2s(stg, iw.base + static_cast<int64_t>(iw.r) * ROUND_BYTES, ROUND_BYTES, &bar[0]);
     }
-    issued = 1;
-    if (++iw.r == iw.A) {
-      iw.r = 0;
-      if (++iw.t < ngw) walk_group(iw, p, lo, warp);
-    }
+    issue(0);
   }
   __syncwarp();
   pdl_launch_dependents();
-  pdl_wait();  // x and y may be the previous launch's
+  pdl_wait();  // x, h and the outputs may be the previous launch's
 
   // ---- x of every matrix this CTA's range touches, [quad c][block b][4]
   // each: requested before the rest of the weights, which would otherwise
   // queue ahead of it
-  const int glast = hi > lo ? mat_of(p, hi - 1) : gfirst;
-  {
+  const int glast = nbc > 0 ? mat_of(p, hi - 1) : gfirst;
+  if (nbc > 0) {
     int xo = 0;
     for (int g = gfirst; g <= glast; ++g) {
       const int K = p.m[g].K;
@@ -251,21 +302,21 @@ __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_co
     }
   }
   cp_async_commit();
+  // ---- the head's h, [row pair c][16-row block b][2]
+  if (HEAD && nhc > 0) {
+    const int nbh = p.hd.K >> 4;
+    for (int i = threadIdx.x; i < (p.hd.K >> 2); i += PW * 32) {
+      const int b = i >> 2, q = i & 3;  // floats 16 b + 4 q .. +3: row pairs 2q, 2q+1
+      const float4 v = __ldg(reinterpret_cast<const float4*>(p.hd.h) + i);
+      *reinterpret_cast<float2*>(hs + ((2 * q) * nbh + b) * 2) = make_float2(v.x, v.y);
+      *reinterpret_cast<float2*>(hs + ((2 * q + 1) * nbh + b) * 2) = make_float2(v.z, v.w);
+    }
+  }
   cp_async_wait_group<0>();
   __syncthreads();
   // ---- the warp's other stages, once x is in: the first round is already
   // here or in flight, so the stream does not stall meanwhile
-  for (int s = 1; s < PST && iw.t < ngw; ++s) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bar[s], ROUND_BYTES);
-      bulk_g2s(stg + s * ROUND_BYTES, iw.base + static_cast<int64_t>(iw.r) * ROUND_BYTES, ROUND_BYTES, &bar[s]);
-    }
-    ++issued;
-    if (++iw.r == iw.A) {
-      iw.r = 0;
-      if (++iw.t < ngw) walk_group(iw, p, lo, warp);
-    }
-  }
+  for (int s = 1; s < PST && iw.t < ngw; ++s) issue(s);
   if (ngw == 0) return;
 
   uint32_t kMagic;  // 0x4B000000 (the bits of 2^23) held in a register
@@ -278,7 +329,73 @@ __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_co
   int xo = 0;  // x offset of matrix g in shared memory
 #pragma unroll 1
   for (int t = 0; t < ngw && ok; ++t) {
-    const int gg = lo + warp + PW * t;
+    const int u = warp + PW * t;
+    if (HEAD && u >= nbc) {
+      // ---------------------------------------------------- a head group
+      const int hg = hlo + u - nbc;
+      const int gsl = p.hd.gsl;
+      const int gs = 1 << gsl;
+      const int A = p.hd.A;
+      const int phase = lane >> gsl;
+      const int pstride = 32 >> gsl;
+      const float* hw = hs + phase * 2;
+      const int hq = (p.hd.K >> 4) * 2;
+      const float2 nbias = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
+      float2 P[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) P[i] = make_float2(0.f, 0.f);
+      float sv[8];
+#pragma unroll 1
+      for (int r = 0; r < A; ++r) {
+        ok = mbar_wait_bounded(&bar[s], par, p.timeout_ns, abort_flag, p.err, K_GEMVR, 3);
+        if (__any_sync(0xffffffffu, !ok)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* st = stg + s * ROUND_BYTES;
+        atom_i8(st, lane, hw + r * pstride * 2, hq, kMagic, nbias, P);
+        if (r == A - 1) {
+          const float4* sp = reinterpret_cast<const float4*>(st + HROUND + (lane & (gs - 1)) * 32);
+          const float4 s0 = sp[0], s1 = sp[1];
+          sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+          sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+        }
+        __syncwarp();
+        if (iw.t < ngw) {  // refill this stage with the round PST ahead
+          if (lane == 0) fence_proxy_async_smem();
+          issue(s);
+        }
+        if (++s == PST) {
+          s = 0;
+          par ^= 1u;
+        }
+      }
+      if (!ok) break;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = P[i].x + P[i].y;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1)
+        if (off >= gs) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+        }
+      const int col = ((hg << gsl) + (lane & (gs - 1))) * 8;
+      if (phase == 0) {
+        float* lp = p.hd.logits + col;
+        if (col + 8 <= p.hd.V) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) lp[i] = acc[i] * sv[i];
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (col + i < p.hd.V) lp[i] = acc[i] * sv[i];
+        }
+      }
+      continue;
+    }
+    // ------------------------------------------------------ a body group
+    const int gg = lo + u;
     while (g < glast && p.m[g + 1].g0 <= gg) {
       xo += p.m[g].K;
       ++g;
@@ -304,16 +421,8 @@ __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_co
       atom_m1(stg + s * ROUND_BYTES, lane, xw + r * pstride * 4, nb * 4, kMagic, acc);
       __syncwarp();
       if (iw.t < ngw) {  // refill this stage with the round PST ahead (the walk is warp-uniform)
-        if (lane == 0) {
-          fence_proxy_async_smem();
-          mbar_arrive_expect_tx(&bar[s], ROUND_BYTES);
-          bulk_g2s(stg + s * ROUND_BYTES, iw.base + static_cast<int64_t>(iw.r) * ROUND_BYTES, ROUND_BYTES, &bar[s]);
-        }
-        ++issued;
-        if (++iw.r == iw.A) {
-          iw.r = 0;
-          if (++iw.t < ngw) walk_group(iw, p, lo, warp);
-        }
+        if (lane == 0) fence_proxy_async_smem();
+        issue(s);
       }
       if (++s == PST) {
         s = 0;
@@ -452,6 +561,11 @@ bool geom_of(int64_t K, int64_t N, RepackGeom* g) {
 
 bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+bool overlaps(const void* a, int64_t abytes, const void* b, int64_t bbytes) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + static_cast<uintptr_t>(bbytes) && b0 < a0 + static_cast<uintptr_t>(abytes);
+}
+
 w4_status launch_repack_like(bool restore, const uint8_t* qw, const float* sc, const uint8_t* zp, const void* wr,
                              int64_t K, int64_t N, uint8_t* qw_out, float* sc_out, uint8_t* zp_out, void* wr_out,
                              cudaStream_t st) {
@@ -502,6 +616,22 @@ w4_status check_rdesc(const w4r_desc& d, RepackGeom* g) {
   return W4_OK;
 }
 
+w4_status check_rdescs(const w4r_desc* descs, int32_t count, int* work) {
+  using namespace w4host;
+  *work = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    RepackGeom g;
+    const w4_status rc = check_rdesc(descs[i], &g);
+    if (rc != W4_OK) {
+      char why[256];
+      snprintf(why, sizeof(why), "%s", w4_last_error());
+      return fail(rc, "descriptor %d: %s", i, why);
+    }
+    if (descs[i].M != 0 && descs[i].N != 0) ++*work;
+  }
+  return W4_OK;
+}
+
 // x floats that CTA c of G must hold: the sum of K over the matrices its
 // range of groups touches.
 int64_t max_x_need(const w4r_desc* d, const RepackGeom* geo, int count, int64_t T, int G) {
@@ -519,21 +649,31 @@ int64_t max_x_need(const w4r_desc* d, const RepackGeom* geo, int count, int64_t 
   return worst;
 }
 
+// CTAs of a launch of T body groups and TH head groups: each CTA takes an
+// equal share of both.
+int grid_of(int64_t T, int64_t TH, const w4host::DeviceInfo& di) {
+  return static_cast<int>(std::min<int64_t>(di.sms, T + TH));
+}
+
+// One launch over the matrices d[0 .. count) and, with hd, the head's TH
+// groups (the caller has checked that the step fits one launch).
 w4_status launch_rgroup(const w4r_desc* d, const RepackGeom* geo, int count, cudaStream_t st,
-                        const w4host::DeviceInfo& di) {
+                        const w4host::DeviceInfo& di, const RHead* hd = nullptr, int32_t TH = 0) {
   using namespace w4host;
   int64_t T = 0;
   for (int i = 0; i < count; ++i) T += geo[i].ngroups;
-  const int G = static_cast<int>(std::min<int64_t>(di.sms, T));
+  if (hd == nullptr) TH = 0;
+  const int G = grid_of(T, TH, di);
   // every CTA stages the x of each matrix its range touches: split the
   // launch until that fits its shared memory
-  if (count > 1 && max_x_need(d, geo, count, T, G) > XCAP) {
+  if (hd == nullptr && count > 1 && max_x_need(d, geo, count, T, G) > XCAP) {
     const int h = count / 2;
     const w4_status rc = launch_rgroup(d, geo, h, st, di);
     if (rc != W4_OK) return rc;
     return launch_rgroup(d + h, geo + h, count - h, st, di);
   }
-  if (T * G >= (int64_t(1) << 31)) return fail(W4_ERR_SHAPE, "too many groups for one launch (%lld)", (long long)T);
+  if ((T + TH) * G >= (int64_t(1) << 31))
+    return fail(W4_ERR_SHAPE, "too many groups for one launch (%lld)", (long long)(T + TH));
   RParams prm;
   std::memset(&prm, 0, sizeof(prm));
   int g0 = 0;
@@ -555,27 +695,32 @@ w4_status launch_rgroup(const w4r_desc* d, const RepackGeom* geo, int count, cud
   }
   prm.count = count;
   prm.T = static_cast<int32_t>(T);
+  prm.TH = TH;
+  if (hd != nullptr) prm.hd = *hd;
   prm.err = di.err;
   prm.timeout_ns = wait_timeout_ns();
-  static int configured[64] = {};
-  if (di.dev < 64 && !configured[di.dev]) {
+  const bool step = hd != nullptr;
+  static int configured[2][64] = {};
+  if (di.dev < 64 && !configured[step][di.dev]) {
     const cudaError_t e =
-        cudaFuncSetAttribute(w4r_gemv_m1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        step ? cudaFuncSetAttribute(w4r_gemv_m1_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_STEP)
+             : cudaFuncSetAttribute(w4r_gemv_m1_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(w4r_gemv)");
-    configured[di.dev] = 1;
+    configured[step][di.dev] = 1;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(G));
   cfg.blockDim = dim3(PW * 32);
-  cfg.dynamicSmemBytes = static_cast<size_t>(SMEM_BYTES);
+  cfg.dynamicSmemBytes = static_cast<size_t>(step ? SMEM_STEP : SMEM_BYTES);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, w4r_gemv_m1_kernel, prm);
-  return e == cudaSuccess ? W4_OK : cuda_fail(e, "launch w4r_gemv");
+  const cudaError_t e = step ? cudaLaunchKernelEx(&cfg, w4r_gemv_m1_kernel<true>, prm)
+                             : cudaLaunchKernelEx(&cfg, w4r_gemv_m1_kernel<false>, prm);
+  return e == cudaSuccess ? W4_OK : cuda_fail(e, step ? "launch w4r_gemv (decode step)" : "launch w4r_gemv");
 }
 
 }  // namespace
@@ -618,16 +763,8 @@ w4_status w4r_matmul_grouped(const w4r_desc* descs, int32_t count, void* stream)
   static thread_local RepackGeom geo[RCAP];
   static thread_local w4r_desc run[RCAP];
   int work = 0;
-  for (int32_t i = 0; i < count; ++i) {
-    RepackGeom g;
-    const w4_status rc = check_rdesc(descs[i], &g);
-    if (rc != W4_OK) {
-      char why[256];
-      snprintf(why, sizeof(why), "%s", w4_last_error());
-      return fail(rc, "descriptor %d: %s", i, why);
-    }
-    if (descs[i].M != 0 && descs[i].N != 0) ++work;
-  }
+  w4_status rc0 = check_rdescs(descs, count, &work);
+  if (rc0 != W4_OK) return rc0;
   if (work == 0) return W4_OK;
   const DeviceInfo* di = nullptr;
   w4_status rc = current_device(&di);
@@ -662,6 +799,77 @@ w4_status w4r_matmul_grouped(const w4r_desc* descs, int32_t count, void* stream)
 w4_status w4r_matmul(const w4r_desc* d, void* stream) {
   if (d == nullptr) return w4host::fail(W4_ERR_NULL, "descriptor is NULL");
   return w4r_matmul_grouped(d, 1, stream);
+}
+
+w4_status w4r_decode_step(const w4r_desc* descs, int32_t count, const float* h, const void* tr, int64_t K, int64_t V,
+                          float* logits, void* stream) {
+  using namespace w4host;
+  if (count < 0) return fail(W4_ERR_SHAPE, "negative count");
+  if (count > 0 && descs == nullptr) return fail(W4_ERR_NULL, "descs is NULL");
+  int work = 0;
+  w4_status rc = count > 0 ? check_rdescs(descs, count, &work) : W4_OK;
+  if (rc != W4_OK) return rc;
+  rc = check_stream_head(h, tr, K, V);
+  if (rc != W4_OK) return rc;
+  if (logits == nullptr) return fail(W4_ERR_NULL, "logits is NULL");
+  if (!aligned_to(logits, 4)) return fail(W4_ERR_ALIGN, "logits must be 4-byte aligned");
+  // h is read when the launch starts and the body's outputs are written
+  // during it: h must not be one of them
+  for (int32_t i = 0; i < count; ++i) {
+    const w4r_desc& d = descs[i];
+    if (d.M != 0 && d.N != 0 && overlaps(h, K * 4, d.y, d.N * 4))
+      return fail(W4_ERR_VALUE, "h overlaps the output of descriptor %d: a step's head reads its input at the start",
+                  i);
+  }
+  const DeviceInfo* di = nullptr;
+  rc = current_device(&di);
+  if (rc != W4_OK) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  static thread_local RepackGeom geo[RCAP];
+  static thread_local w4r_desc run[RCAP];
+  int n = 0;
+  bool one_launch = work <= RCAP && K <= HKS;
+  for (int32_t i = 0; i < count && one_launch; ++i) {
+    const w4r_desc& d = descs[i];
+    if (d.M == 0 || d.N == 0 || d.K == 0) continue;
+    geom_of(d.K, d.N, &geo[n]);
+    run[n++] = d;
+  }
+  StreamHeadGeom hg;
+  stream_head_geom(K, V, &hg);
+  if (one_launch && n > 0) {
+    int64_t T = 0;
+    for (int i = 0; i < n; ++i) T += geo[i].ngroups;
+    one_launch = max_x_need(run, geo, n, T, grid_of(T, hg.ngroups, *di)) <= XCAP;
+  }
+  if (!one_launch) {
+    // more matrices, x or h than one launch holds: the body's launches, then the head's
+    rc = w4r_matmul_grouped(descs, count, stream);
+    if (rc != W4_OK) return rc;
+    return launch_stream_head(h, tr, K, V, logits, st, *di);
+  }
+  for (int32_t i = 0; i < count; ++i) {  // K = 0: y is the epilogue of 0
+    const w4r_desc& d = descs[i];
+    if (d.M == 0 || d.N == 0 || d.K != 0) continue;
+    w4_desc z = {};
+    z.bias = d.bias;
+    z.residual = d.residual;
+    z.ldr = d.ldr;
+    z.act = d.act;
+    rc = launch_zero_fill(d.y, d.N, 1, d.N, st, &z);
+    if (rc != W4_OK) return rc;
+  }
+  if (n == 0) return launch_stream_head(h, tr, K, V, logits, st, *di);
+  RHead hd;
+  hd.tr = static_cast<const uint8_t*>(tr);
+  hd.h = h;
+  hd.logits = logits;
+  hd.group_bytes = hg.group_bytes;
+  hd.K = static_cast<int32_t>(K);
+  hd.V = static_cast<int32_t>(V);
+  hd.gsl = hg.gsl;
+  hd.A = hg.A;
+  return launch_rgroup(run, geo, n, st, *di, &hd, hg.ngroups);
 }
 
 }  // extern "C"

@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol():
 def test_abi_version_and_status_strings():
     lib = _lib()
     from int8_weight_quantized_w4_b200 import _lib as L
-    assert lib.w4_abi_version() == L.ABI_VERSION == 5
+    assert lib.w4_abi_version() == L.ABI_VERSION == 6
     assert lib.w4_status_string(0) == b"W4_OK"
     assert lib.w4_status_string(6) == b"W4_ERR_TIMEOUT"
     assert lib.w4_status_string(99) == b"W4_ERR_UNKNOWN"
