@@ -241,7 +241,7 @@ W4_API w4_status w4_repack_restore(const void* wr, int64_t K, int64_t N, uint8_t
 /* One decode matmul on a repacked weight: y[1, N] = act(x[1, K] . W + bias)
  * + residual, the fields and the epilogue as in w4_desc (ldx / ldy / ldr are
  * not used: one row). Requires M == 1 (W4_ERR_SHAPE otherwise), K % 32 == 0,
- * K <= 8192, N % 8 == 0, x and wr 16-byte aligned, y / bias / residual
+ * K <= 14336, N % 8 == 0, x and wr 16-byte aligned, y / bias / residual
  * 4-byte aligned. No workspace: every output column is summed inside one
  * warp. reserved must be 0. */
 typedef struct w4r_desc {
@@ -261,7 +261,8 @@ typedef struct w4r_desc {
 } w4r_desc;
 
 /* Many independent decode matmuls on repacked weights in as few launches as
- * possible (64 per launch). `descs` is a HOST array read during the call
+ * possible (128 per launch; a launch whose CTAs would each stage more than
+ * 14336 floats of x is split). `descs` is a HOST array read during the call
  * only; outputs must not overlap each other or any input. The launch lets the
  * next launch on the stream begin streaming its weights while this one
  * finishes (programmatic dependent launch); x is read and y written only
@@ -430,7 +431,7 @@ W4_API w4_status i8r_head_argmax(const float* h, const void* tr, int64_t K, int6
  * - h, tr, K, V, logits: as for i8r_head_logits. h is read when the launch
  *   starts, so it must not overlap any y of `descs` (W4_ERR_VALUE): within a
  *   step the head's input is not one of the body's outputs.
- * - A step that one launch cannot hold (more than 64 weights, K of the head
+ * - A step that one launch cannot hold (more than 128 weights, K of the head
  *   above 2048, or more x than a CTA stages) runs as the body's launches
  *   followed by the head's, with the same results.
  * - The launch starts streaming while the previous work on the stream

@@ -45,7 +45,7 @@
 //  * The CTA stages the x of every matrix its share touches in shared memory
 //    as [row quad c][block b][4 floats], so lanes reading different blocks hit
 //    different banks (the host splits a launch whose shares would need more
-//    than 8192 floats).
+//    than 14336 floats).
 //  * The launch lets the next launch in the stream start early (programmatic
 //    dependent launch): a CTA requests its first rounds before it waits for
 //    the previous launch to finish, and reads x / writes y only after that
@@ -78,16 +78,21 @@ constexpr int SC_BYTES = 1024;
 constexpr int ROUND_WORDS = ROUND_BYTES / 4;  // 1312
 constexpr int PW = 16;                        // warps per CTA, each its own stream
 constexpr int PST = 2;                        // stages per warp
-constexpr int RCAP = 64;                      // matrices per launch
-constexpr int XCAP = 8192;                    // floats of x a CTA can hold
+constexpr int RCAP = 128;                     // matrices per launch
+// floats of x a CTA can hold: 14336 takes any three consecutive matrices of
+// a stack with K up to 3072, 3072 and 8192 (the range of a CTA over a
+// 128-matrix launch touches at most three), so such a stack is one launch
+constexpr int XCAP = 14336;
+constexpr int XCAP_STEP = 12288;              // the same in the fused step, whose CTA also holds h
 constexpr int STAGE_SMEM = PW * PST * ROUND_BYTES;
 constexpr int SMEM_BYTES = STAGE_SMEM + XCAP * 4 + PW * PST * 8 + PW * 4;
 // the fused decode step: the head's rounds share the stages, its h follows
 constexpr int HROUND = w4host::kStreamHeadRound;  // table bytes of a head round
 constexpr int HKS = 2048;                         // rows of the head's h a CTA of the step holds
-constexpr int SMEM_STEP = SMEM_BYTES + HKS * 4;
+constexpr int SMEM_STEP = STAGE_SMEM + XCAP_STEP * 4 + PW * PST * 8 + PW * 4 + HKS * 4;
 static_assert(HROUND + 32 * 32 <= ROUND_BYTES, "a head round and its scales fit a stage");
-static_assert(SMEM_BYTES % 16 == 0 && SMEM_STEP <= 227 * 1024, "shared memory of one CTA");
+static_assert(SMEM_BYTES <= 227 * 1024 && SMEM_STEP <= 227 * 1024, "shared memory of one CTA");
+static_assert((STAGE_SMEM + XCAP_STEP * 4 + PW * PST * 8 + PW * 4) % 16 == 0, "h 16-byte aligned");
 
 struct RMat {
   const uint8_t* wr;
@@ -235,11 +240,13 @@ __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_co
   const int units = nbc + nhc;
   const int ngw = units > warp ? (units - warp + PW - 1) / PW : 0;  // units of this warp
 
+  constexpr int XC = HEAD ? XCAP_STEP : XCAP;
   uint8_t* stg = smem + warp * (PST * ROUND_BYTES);
   float* xs = reinterpret_cast<float*>(smem + STAGE_SMEM);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + STAGE_SMEM + XCAP * 4) + warp * PST;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + STAGE_SMEM + XCAP * 4 + PW * PST * 8) + warp;
-  float* hs = reinterpret_cast<float*>(smem + SMEM_BYTES);  // the head's h (fused step only)
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + STAGE_SMEM + XC * 4) + warp * PST;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + STAGE_SMEM + XC * 4 + PW * PST * 8) + warp;
+  // the head's h (fused step only)
+  float* hs = reinterpret_cast<float*>(smem + STAGE_SMEM + XC * 4 + PW * PST * 8 + PW * 4);
 
   // ---- x into L2 now: a cache hint only (the values are read after the
   // wait), so that the staging below does not queue behind weight bytes
@@ -840,7 +847,7 @@ w4_status w4r_decode_step(const w4r_desc* descs, int32_t count, const float* h, 
   if (one_launch && n > 0) {
     int64_t T = 0;
     for (int i = 0; i < n; ++i) T += geo[i].ngroups;
-    one_launch = max_x_need(run, geo, n, T, grid_of(T, hg.ngroups, *di)) <= XCAP;
+    one_launch = max_x_need(run, geo, n, T, grid_of(T, hg.ngroups, *di)) <= XCAP_STEP;
   }
   if (!one_launch) {
     // more matrices, x or h than one launch holds: the body's launches, then the head's

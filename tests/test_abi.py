@@ -224,7 +224,7 @@ def _rdesc(**kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(M=2), 2), (dict(N=60), 2), (dict(K=40), 2), (dict(K=8224), 2), (dict(M=-1), 2),
+    (dict(M=2), 2), (dict(N=60), 2), (dict(K=40), 2), (dict(K=14368), 2), (dict(M=-1), 2),
     (dict(x=0x1004), 3), (dict(wr=0x2008), 3), (dict(y=0x5002), 3), (dict(bias=0x6002), 3),
     (dict(x=0), 1), (dict(wr=0), 1), (dict(y=0), 1), (dict(act=5), 8), (dict(reserved=1), 8),
 ])

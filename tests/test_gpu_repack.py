@@ -128,6 +128,39 @@ def test_gpt2_decode_stack_grouped_on_repacked_weights():
         assert T.equal(a_, it["y"]), "not run-to-run deterministic"
 
 
+def test_dense38_stack_in_one_launch_sampled():
+    """The 128 weights of the 3.8B-shaped stack (K up to 8192) as one grouped
+    call: one launch (every CTA's x fits its shared memory). The four layer
+    weights are generated once and shared by the 32 layers' descriptors, each
+    with its own x and y; 16 columns of every output are checked against the
+    oracle on the same columns of the page-format buffers."""
+    T = torch()
+    shapes = synth.DENSE38_LAYER_SHAPES
+    Ws = [synth.w4_weight(K, N, 300 + i) for i, (_, K, N) in enumerate(shapes)]
+    wrs = [_repacked(W)[1] for W in Ws]
+    items, host = [], []
+    for layer in range(synth.DENSE38_LAYERS):
+        for i, (_, K, N) in enumerate(shapes):
+            x = synth.activations(1, K, 400 + 4 * layer + i)
+            items.append({"x": dev(x), "wr": wrs[i], "y": T.full((1, N), float("nan"), device="cuda"), "K": K, "N": N})
+            host.append((i, x))
+    assert len(items) == 128
+    w4().w4r_matmul_grouped(items)
+    T.cuda.synchronize()
+    g = np.random.default_rng(5)
+    for (i, x), it in zip(host, items):
+        W = Ws[i]
+        K, N = W["K"], W["N"]
+        y = it["y"].cpu().numpy()
+        assert np.all(np.isfinite(y))
+        for c0 in sorted(set([0, N - 8] + [int(v) * 8 for v in g.integers(0, N // 8, 2)])):
+            qw = np.ascontiguousarray(W["qw"].reshape(K, N // 2)[:, c0 // 2:c0 // 2 + 4])
+            sc = np.ascontiguousarray(W["scales"].reshape(K // 32, N)[:, c0:c0 + 8])
+            zp = np.ascontiguousarray(W["zp"].reshape(K // 32, N // 2)[:, c0 // 2:c0 // 2 + 4])
+            y_ref, a = oracle.w4_matmul_ref(x, qw, sc, zp, K, 8)
+            check(y[:, c0:c0 + 8], y_ref, a, f"3.8B weight {i} K={K} N={N} columns {c0}..{c0 + 7}")
+
+
 def _exact_r(q, zp, s, x):
     K, N = q.shape
     qw, sc, zpk = pins.make_w4(q, zp, s)
