@@ -440,6 +440,16 @@ W4_API w4_status i8r_head_argmax(const float* h, const void* tr, int64_t K, int6
 W4_API w4_status w4r_decode_step(const w4r_desc* descs, int32_t count, const float* h, const void* tr, int64_t K,
                                  int64_t V, float* logits, void* stream);
 
+/* The same step with greedy decoding instead of the logits (as
+ * i8r_head_argmax): *token = argmax_v of exactly the logits w4r_decode_step
+ * computes (ties to the lowest id; -0 equals +0), *best_logit (may be NULL)
+ * = that logit; the logits are not written. keys: 8 bytes of device memory
+ * (8-byte aligned) that the call clears and uses. One launch for the step
+ * and one small launch that turns the key into the token. */
+W4_API w4_status w4r_decode_step_argmax(const w4r_desc* descs, int32_t count, const float* h, const void* tr,
+                                        int64_t K, int64_t V, int32_t* token, float* best_logit, void* keys,
+                                        void* stream);
+
 /* The tile layout of the int8 head, read by the tensor-core head
  * (i8t_head_logits / i8t_head_argmax) for 1 to 8 last-position rows. The
  * page's table bytes and scales ("ONNX export, quantization and the browser

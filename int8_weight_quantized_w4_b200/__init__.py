@@ -444,6 +444,20 @@ def w4r_decode_step(items: Sequence[dict] | None, h, tr, K: int, V: int, logits=
     return logits
 
 
+def w4r_decode_step_argmax(items: Sequence[dict] | None, h, tr, K: int, V: int, descs=None, stream=None):
+    """One decode step in one launch with greedy decoding: the matmuls of
+    `items` and (token int32 [1], best logit fp32 [1]) of h on the head."""
+    torch = _torch()
+    if descs is None:
+        descs = make_rdescs(items or [])
+    tok = torch.empty(1, dtype=torch.int32, device=h.device)
+    best = torch.empty(1, dtype=torch.float32, device=h.device)
+    keys = torch.empty(1, dtype=torch.int64, device=h.device)
+    _check(lib().w4r_decode_step_argmax(descs, len(descs), _ptr(h), _ptr(tr), K, V, _ptr(tok), _ptr(best), _ptr(keys),
+                                        _stream_handle(stream)), "w4r_decode_step_argmax")
+    return tok, best
+
+
 def i8r_head_argmax(h, tr, K: int, V: int, stream=None):
     """(token int32 [1], best logit fp32 [1]) of one row h on a repacked head."""
     torch = _torch()

@@ -105,6 +105,8 @@ SIGNATURES = {
     "i8r_head_logits": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),
     "w4r_decode_step": (C.c_int, [C.POINTER(W4RDesc), C.c_int32, C.c_void_p, C.c_void_p, C.c_int64, C.c_int64,
                                   C.c_void_p, C.c_void_p]),
+    "w4r_decode_step_argmax": (C.c_int, [C.POINTER(W4RDesc), C.c_int32, C.c_void_p, C.c_void_p, C.c_int64,
+                                         C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "i8t_head_repacked_bytes": (C.c_size_t, [C.c_int64, C.c_int64]),
     "i8t_head_repack": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),
     "i8t_head_repack_restore": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_int64, C.c_void_p,

@@ -115,7 +115,8 @@ struct RMat {
 struct RHead {
   const uint8_t* tr;
   const float* h;
-  float* logits;
+  float* logits;              // or nullptr: greedy decoding into keys
+  unsigned long long* keys;   // the 64-bit (logit, token) key of the maximum
   int64_t group_bytes;
   int32_t K, V, gsl, A;
 };
@@ -388,7 +389,17 @@ __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_co
           for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
         }
       const int col = ((hg << gsl) + (lane & (gs - 1))) * 8;
-      if (phase == 0) {
+      if (p.hd.keys != nullptr) {
+        unsigned long long best = 0ull;
+        if (phase == 0) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (col + i < p.hd.V) best = max(best, head_key(acc[i] * sv[i], static_cast<uint32_t>(col + i)));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+        if (lane == 0 && best != 0ull) atomicMax(p.hd.keys, best);
+      } else if (phase == 0) {
         float* lp = p.hd.logits + col;
         if (col + 8 <= p.hd.V) {
 #pragma unroll
@@ -808,8 +819,13 @@ w4_status w4r_matmul(const w4r_desc* d, void* stream) {
   return w4r_matmul_grouped(d, 1, stream);
 }
 
-w4_status w4r_decode_step(const w4r_desc* descs, int32_t count, const float* h, const void* tr, int64_t K, int64_t V,
-                          float* logits, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The step with the head's logits (keys == nullptr) or its greedy token.
+w4_status decode_step(const w4r_desc* descs, int32_t count, const float* h, const void* tr, int64_t K, int64_t V,
+                      float* logits, unsigned long long* keys, int32_t* token, float* best_logit, void* stream) {
   using namespace w4host;
   if (count < 0) return fail(W4_ERR_SHAPE, "negative count");
   if (count > 0 && descs == nullptr) return fail(W4_ERR_NULL, "descs is NULL");
@@ -818,8 +834,15 @@ w4_status w4r_decode_step(const w4r_desc* descs, int32_t count, const float* h, 
   if (rc != W4_OK) return rc;
   rc = check_stream_head(h, tr, K, V);
   if (rc != W4_OK) return rc;
-  if (logits == nullptr) return fail(W4_ERR_NULL, "logits is NULL");
-  if (!aligned_to(logits, 4)) return fail(W4_ERR_ALIGN, "logits must be 4-byte aligned");
+  if (keys == nullptr) {
+    if (logits == nullptr) return fail(W4_ERR_NULL, "logits is NULL");
+    if (!aligned_to(logits, 4)) return fail(W4_ERR_ALIGN, "logits must be 4-byte aligned");
+  } else {
+    if (V > 0x7fffffff) return fail(W4_ERR_SHAPE, "V must be below 2^31");
+    if (token == nullptr) return fail(W4_ERR_NULL, "token is NULL");
+    if (!aligned_to(token, 4) || !aligned_to(best_logit, 4) || !aligned_to(keys, 8))
+      return fail(W4_ERR_ALIGN, "token / best 4-byte, keys 8-byte aligned");
+  }
   // h is read when the launch starts and the body's outputs are written
   // during it: h must not be one of them
   for (int32_t i = 0; i < count; ++i) {
@@ -832,6 +855,11 @@ w4_status w4r_decode_step(const w4r_desc* descs, int32_t count, const float* h, 
   rc = current_device(&di);
   if (rc != W4_OK) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the head alone (logits or greedy token), stream-ordered after the body
+  auto head = [&]() -> w4_status {
+    if (keys == nullptr) return launch_stream_head(h, tr, K, V, logits, st, *di);
+    return i8r_head_argmax(h, tr, K, V, token, best_logit, keys, stream);
+  };
   static thread_local RepackGeom geo[RCAP];
   static thread_local w4r_desc run[RCAP];
   int n = 0;
@@ -853,7 +881,7 @@ w4_status w4r_decode_step(const w4r_desc* descs, int32_t count, const float* h, 
     // more matrices, x or h than one launch holds: the body's launches, then the head's
     rc = w4r_matmul_grouped(descs, count, stream);
     if (rc != W4_OK) return rc;
-    return launch_stream_head(h, tr, K, V, logits, st, *di);
+    return head();
   }
   for (int32_t i = 0; i < count; ++i) {  // K = 0: y is the epilogue of 0
     const w4r_desc& d = descs[i];
@@ -866,17 +894,40 @@ w4_status w4r_decode_step(const w4r_desc* descs, int32_t count, const float* h, 
     rc = launch_zero_fill(d.y, d.N, 1, d.N, st, &z);
     if (rc != W4_OK) return rc;
   }
-  if (n == 0) return launch_stream_head(h, tr, K, V, logits, st, *di);
+  if (n == 0) return head();
   RHead hd;
   hd.tr = static_cast<const uint8_t*>(tr);
   hd.h = h;
-  hd.logits = logits;
+  hd.logits = keys == nullptr ? logits : nullptr;
+  hd.keys = keys;
   hd.group_bytes = hg.group_bytes;
   hd.K = static_cast<int32_t>(K);
   hd.V = static_cast<int32_t>(V);
   hd.gsl = hg.gsl;
   hd.A = hg.A;
-  return launch_rgroup(run, geo, n, st, *di, &hd, hg.ngroups);
+  if (keys != nullptr) {
+    const cudaError_t e = cudaMemsetAsync(keys, 0, 8, st);
+    if (e != cudaSuccess) return cuda_fail(e, "clear argmax key");
+  }
+  rc = launch_rgroup(run, geo, n, st, *di, &hd, hg.ngroups);
+  if (rc != W4_OK || keys == nullptr) return rc;
+  return launch_argmax_finish(keys, 1, token, best_logit, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+w4_status w4r_decode_step(const w4r_desc* descs, int32_t count, const float* h, const void* tr, int64_t K, int64_t V,
+                          float* logits, void* stream) {
+  return decode_step(descs, count, h, tr, K, V, logits, nullptr, nullptr, nullptr, stream);
+}
+
+w4_status w4r_decode_step_argmax(const w4r_desc* descs, int32_t count, const float* h, const void* tr, int64_t K,
+                                 int64_t V, int32_t* token, float* best_logit, void* keys, void* stream) {
+  if (keys == nullptr) return w4host::fail(W4_ERR_NULL, "keys is NULL");
+  return decode_step(descs, count, h, tr, K, V, nullptr, static_cast<unsigned long long*>(keys), token, best_logit,
+                     stream);
 }
 
 }  // extern "C"

@@ -203,3 +203,45 @@ def test_refusals():
     bad["x"] = dev(synth.activations(2, 64, 1))
     with pytest.raises(w4().W4Error):  # M = 2 in the body
         w4().w4r_decode_step([bad], dev(synth.activations(1, K, 1)), tr, K, V)
+
+
+@pytest.mark.parametrize("K,V,tag", [(768, 50257, 1), (64, 1000, 2), (4096, 777, 3)])
+def test_greedy_step_is_the_argmax_of_the_step_logits(K, V, tag):
+    """The greedy step returns the token and logit of exactly the fused
+    step's logits (ties to the lowest id), and the body outputs of the
+    logits step; K = 4096 takes the two-launch form."""
+    T = torch()
+    shapes = [(K2, N) for _, K2, N in synth.gpt2_stack_shapes()][:6]
+    host, items = _body(shapes, tag0=100 + tag)
+    H, tr = _head(K, V, tag)
+    h_host = synth.activations(1, K, 200 + tag)
+    h = dev(h_host)
+    lg = w4().w4r_decode_step(items, h, tr, K, V)
+    T.cuda.synchronize()
+    ys = [it["y"].clone() for it in items]
+    for it in items:
+        it["y"].fill_(float("nan"))
+    tok, best = w4().w4r_decode_step_argmax(items, h, tr, K, V)
+    T.cuda.synchronize()
+    l = lg.cpu().numpy()[0]
+    assert int(tok.item()) == int(np.argmax(l)) and float(best.item()) == float(l.max())
+    for a, it in zip(ys, items):
+        assert T.equal(a, it["y"])
+    ref, a = oracle.i8_head_ref(h_host, H["table"], H["scales"], K, V, H["ldt"])
+    rtok, _, _ = oracle.i8_head_argmax_ref(h_host, H["table"], H["scales"], K, V, H["ldt"])
+    g = int(tok.item())
+    assert g == int(rtok[0]) or ref[0, g] >= ref[0, int(rtok[0])] - 2 * oracle.tolerance(a)[0, int(rtok[0])]
+
+
+def test_greedy_step_ties_and_signed_zero():
+    K, V = 32, 1000
+    table = np.full((K, V), -20, np.int8)
+    table[:, 123] = 0
+    table[:, 700] = 0
+    s = np.full(V, 0.5, np.float32)
+    s[123] = -0.5  # 0 * -0.5 = -0, equal to the +0 of column 700
+    tr = w4().i8_head_repack(dev(table), dev(s), K, V)
+    host, items = _body([(64, 64)], tag0=120)
+    tok, best = w4().w4r_decode_step_argmax(items, dev(np.ones((1, K), np.float32)), tr, K, V)
+    torch().cuda.synchronize()
+    assert int(tok.item()) == 123 and float(best.item()) == 0.0
