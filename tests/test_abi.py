@@ -235,6 +235,34 @@ def test_w4r_argument_errors_before_any_launch(kw, status):
     assert lib.w4_last_error()
 
 
+def test_decode_step_argument_errors_before_any_launch():
+    """The one-launch step checks its body descriptors, its head and the
+    aliasing of h with the body's outputs on the host: every refusal here
+    comes before the device is touched."""
+    lib = _lib()
+    from int8_weight_quantized_w4_b200._lib import W4RDesc
+    good = (W4RDesc * 1)(_rdesc())
+    h, tr, lg, K, V = 0x9000, 0xA000, 0xB000, 64, 100
+    step = lib.w4r_decode_step
+    assert step(good, 1, h, tr, K, V, 0, None) == 1          # logits NULL
+    assert step(good, 1, h, tr, K, V, 0xB002, None) == 3     # logits misaligned
+    assert step(good, 1, 0x9004, tr, K, V, lg, None) == 3    # h not 16-byte aligned
+    assert step(good, 1, h, 0xA008, K, V, lg, None) == 3     # table not 16-byte aligned
+    assert step(good, 1, h, tr, 72, V, lg, None) == 2        # head K % 16 != 0
+    assert step(good, 1, 0, tr, K, V, lg, None) == 1         # h NULL
+    assert step(good, -1, h, tr, K, V, lg, None) == 2        # negative count
+    assert step(None, 1, h, tr, K, V, lg, None) == 1         # descs NULL
+    bad = (W4RDesc * 1)(_rdesc(M=2))
+    assert step(bad, 1, h, tr, K, V, lg, None) == 2          # a body descriptor's own check
+    # h inside the body's output y (0x5000 .. 0x5100): refused
+    assert step(good, 1, 0x5040, tr, K, V, lg, None) == 8
+    assert b"overlaps" in lib.w4_last_error()
+    argmax = lib.w4r_decode_step_argmax
+    assert argmax(good, 1, h, tr, K, V, 0xC000, 0, 0, None) == 1        # keys NULL
+    assert argmax(good, 1, h, tr, K, V, 0, 0, 0xD000, None) == 1        # token NULL
+    assert argmax(good, 1, h, tr, K, V, 0xC000, 0, 0xD004, None) == 3   # keys misaligned
+
+
 def test_w4r_noops_and_repack_shape_errors_need_no_device():
     lib = _lib()
     assert lib.w4r_matmul(C.byref(_rdesc(M=0)), None) == 0
