@@ -741,6 +741,10 @@ def config3(peaks, budget, wl):
                                  n, el)}
 
 
+def _scaled(v, k):
+    return None if v is None else int(v) * k
+
+
 def config4(peaks, budget, clocks):
     """3.8B-dense-shaped stack, 32 layers x [3072x9216, 3072x3072, 3072x16384,
     8192x3072]: decode at M = 1 (streaming layout), 8 (split-K GEMV) and 32
@@ -779,7 +783,10 @@ def config4(peaks, budget, clocks):
                         "ms_per_step": round(ms1, 4), "tokens_per_s": round(1e3 / ms1, 1),
                         "roofline": {"kernel": "w4r_gemv_m1_kernel", "bound": "hbm", "achieved": round(g1, 1),
                                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                     "frac": round(g1 / peaks["hbm_gbs"], 4)}}
+                                     "frac": round(g1 / peaks["hbm_gbs"], 4),
+                                     "traffic": _scaled(profiled_traffic("w4r_gemv_3p8b_4layers_m1.md"), 8),
+                                     "traffic_note": "ncu DRAM bytes of 4 of the 32 layers (one launch of 16 weights) "
+                                                     "x 8: the traffic grows with the layers streamed"}}
     # the tile layout of the 128 weights, for M = 32 and the prefill
     wts = [w4.w4t_repack(Wd["qw"], Wd["scales"], Wd["zp"], K, N) for Wd, (K, N) in zip(weights, shapes)]
 
@@ -806,7 +813,9 @@ def config4(peaks, budget, clocks):
         pk = fp32_alu_peak_tflops(clocks.get("sm_mhz"))
         roof = {"kernel": "w4_gemv_kernel<8> (split-K GEMV)", "bound": "alu", "achieved": round(tfl, 2),
                 "peak": round(pk, 1), "unit": "TFLOP/s", "frac": round(tfl / pk, 4),
-                "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x the sampled SM clock"}
+                "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x the sampled SM clock",
+                "traffic": _scaled(profiled_traffic("w4_gemv_pageformat_3p8b_4layers_m8.md"), 8),
+                "traffic_note": "ncu DRAM bytes of 4 of the 32 layers x 8"}
         out[f"decode_M{M}"] = {"metric": "TFLOP/s (algorithmic 2MKN)", "value": round(tfl, 2), "unit": "TFLOP/s",
                                "weight_GB_per_s": round(gb, 1), "ms_per_step": round(msm, 4), "roofline": roof}
         del xm, ym, items, descs, ws
@@ -978,7 +987,10 @@ def profile_case(name: str, calls: int) -> None:
     """Run one workload's kernels `calls` times (no timing, no output but one
     line) so that a profiler can capture them: "step" (the decode step in one
     launch: the 48 GPT-2 weights and the head, streaming layouts, M = 1),
-    "body" (the 48 GPT-2 weights in the streaming layout, M = 1), "head" (the int8 head, streaming
+    "body" (the 48 GPT-2 weights in the streaming layout, M = 1),
+    "decode-3p8b" / "decode-3p8b-m8" (four layers of the 3.8B-shaped stack, 16
+    weights, 290 MB: the streaming GEMV at M = 1, the page-format split-K
+    GEMV at M = 8), "head" (the int8 head, streaming
     layout, M = 1), "head-tile" / "head-tile-m8" (the int8 head in the tile
     layout, tensor cores, M = 1 / 8), "prefill-gpt2" (the 48 weights in the tile layout at
     M = 58), "prefill-3p8b" (one 3.8B-shaped layer, 4 weights in the tile
@@ -1013,6 +1025,30 @@ def profile_case(name: str, calls: int) -> None:
             scratch = torch.empty(max(w4.w4t_workspace_size(descs), 16), dtype=torch.uint8, device=dev)
             run = lambda: _ok(lib.w4t_matmul_grouped(descs, len(descs), scratch.data_ptr(), scratch.numel(), hs), lib,
                               "w4t")
+    elif name in ("decode-3p8b", "decode-3p8b-m8"):
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(synth.BASE_SEED + 38)
+        M = 8 if name.endswith("m8") else 1
+        items = []
+        for _, K, N in synth.dense38_stack_shapes()[:16]:
+            qw = torch.randint(0, 256, (K * N // 2,), dtype=torch.uint8, device=dev, generator=gen)
+            sc = torch.empty((K // 32, N), device=dev).uniform_(0.005, 0.02, generator=gen)
+            zp = torch.randint(0, 256, (K // 32 * N // 2,), dtype=torch.uint8, device=dev, generator=gen)
+            it = {"x": torch.randn((M, K), device=dev, generator=gen), "y": torch.empty((M, N), device=dev), "K": K,
+                  "N": N}
+            if M == 1:
+                it["wr"] = w4.w4_repack(qw, sc, zp, K, N)
+            else:
+                it.update({"qw": qw, "scales": sc, "zp": zp})
+            items.append(it)
+        if M == 1:
+            descs = w4.make_rdescs(items)
+            run = lambda: _ok(lib.w4r_matmul_grouped(descs, len(descs), hs), lib, "w4r")
+        else:
+            descs = w4.make_descs(items)
+            ws = torch.zeros(max(w4.w4_matmul_grouped_workspace_size(descs), 16), dtype=torch.uint8, device=dev)
+            run = lambda: _ok(lib.w4_matmul_grouped(descs, len(descs), ws.data_ptr(), ws.numel(), hs), lib,
+                              "w4_matmul_grouped")
     elif name in ("head-tile", "head-tile-m8"):
         H = synth.i8_head(HEAD_K, HEAD_V)
         tt = w4.i8t_head_repack(torch.from_numpy(H["table"]).to(dev), torch.from_numpy(H["scales"]).to(dev),
@@ -1050,7 +1086,7 @@ def main():
                     help="device seconds of the timed step replays (the body and head alone get half each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config measurements (configs 0, 2, 3, 4)")
-    ap.add_argument("--profile-case", choices=["step", "body", "head", "head-tile", "head-tile-m8", "prefill-gpt2", "prefill-3p8b"],
+    ap.add_argument("--profile-case", choices=["step", "body", "decode-3p8b", "decode-3p8b-m8", "head", "head-tile", "head-tile-m8", "prefill-gpt2", "prefill-3p8b"],
                     default=None,
                     help="only run one workload's kernels a few times, for a profiler (see profiles/)")
     ap.add_argument("--calls", type=int, default=4, help="calls of --profile-case")

@@ -30,8 +30,10 @@
 //   multiple of 8 gs) are zero in the repacked buffer and never written.
 //
 // GEMV design (sm_100a, M = 1):
-//  * One persistent CTA per SM takes an equal share of the launch's groups
-//    (all matrices' groups in one flat list; CTA c takes [c T / G, (c+1) T / G)).
+//  * One persistent CTA per SM takes a contiguous share of the launch's groups
+//    (all matrices' groups in one flat list), cut by the host so that every
+//    CTA streams about the same number of rounds (a group is nb gs / 32
+//    rounds: 3 for K = 3072, 8 for K = 8192).
 //    Each of its 16 warps is an independent stream: warp w owns the groups
 //    lo + w, lo + w + 16, ... of that share, so every output column is summed
 //    inside one warp, with no partial sums in memory and no workspace. For
@@ -121,12 +123,17 @@ struct RHead {
   int32_t K, V, gsl, A;
 };
 
+constexpr int GMAX = 256;  // CTAs of a launch at most
+
 struct RParams {
   RMat m[RCAP];
   int32_t count;
   int32_t T;   // body groups of the launch
   int32_t TH;  // head groups (the fused step; 0 otherwise)
   RHead hd;
+  // body groups of CTA c: [cfirst[c], cfirst[c + 1]), cut so that every CTA
+  // streams about the same number of rounds (groups of a large K have more)
+  int32_t cfirst[GMAX + 1];
   ErrorWord* err;
   uint64_t timeout_ns;
 };
@@ -233,8 +240,8 @@ __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_co
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = gridDim.x;
-  const int lo = range_lo(blockIdx.x, p.T, G);
-  const int hi = range_lo(blockIdx.x + 1, p.T, G);
+  const int lo = p.cfirst[blockIdx.x];
+  const int hi = p.cfirst[blockIdx.x + 1];
   const int nbc = hi - lo;  // body groups of this CTA
   const int hlo = HEAD ? range_lo(blockIdx.x, p.TH, G) : 0;
   const int nhc = HEAD ? range_lo(blockIdx.x + 1, p.TH, G) - hlo : 0;  // head groups of this CTA
@@ -652,12 +659,30 @@ w4_status check_rdescs(const w4r_desc* descs, int32_t count, int* work) {
 
 // x floats that CTA c of G must hold: the sum of K over the matrices its
 // range of groups touches.
-int64_t max_x_need(const w4r_desc* d, const RepackGeom* geo, int count, int64_t T, int G) {
+// cfirst[0 .. G]: CTA c takes body groups [cfirst[c], cfirst[c + 1]), the
+// first group whose rounds before it reach c R / G of the launch's R rounds.
+void split_by_rounds(const RepackGeom* geo, int count, int G, int32_t* cfirst) {
+  int64_t R = 0;
+  for (int i = 0; i < count; ++i) R += static_cast<int64_t>(geo[i].ngroups) * geo[i].A;
+  int64_t g0 = 0, r0 = 0;  // groups and rounds before matrix i
+  int i = 0;
+  for (int c = 0; c <= G; ++c) {
+    const int64_t t = c * R / G;
+    while (i < count && r0 + static_cast<int64_t>(geo[i].ngroups) * geo[i].A < t) {
+      r0 += static_cast<int64_t>(geo[i].ngroups) * geo[i].A;
+      g0 += geo[i].ngroups;
+      ++i;
+    }
+    cfirst[c] = static_cast<int32_t>(i < count ? g0 + (t - r0 + geo[i].A - 1) / geo[i].A : g0);
+  }
+}
+
+int64_t max_x_need(const w4r_desc* d, const RepackGeom* geo, int count, const int32_t* cfirst, int G) {
   int64_t worst = 0;
   int64_t g0 = 0;
   int gi = 0;
   for (int c = 0; c < G; ++c) {
-    const int64_t lo = c * T / G, hi = (c + 1) * T / G;
+    const int64_t lo = cfirst[c], hi = cfirst[c + 1];
     if (hi <= lo) continue;
     while (gi + 1 < count && g0 + geo[gi].ngroups <= lo) g0 += geo[gi++].ngroups;
     int64_t need = 0, gg0 = g0;
@@ -670,7 +695,7 @@ int64_t max_x_need(const w4r_desc* d, const RepackGeom* geo, int count, int64_t 
 // CTAs of a launch of T body groups and TH head groups: each CTA takes an
 // equal share of both.
 int grid_of(int64_t T, int64_t TH, const w4host::DeviceInfo& di) {
-  return static_cast<int>(std::min<int64_t>(di.sms, T + TH));
+  return static_cast<int>(std::min<int64_t>(std::min(di.sms, GMAX), T + TH));
 }
 
 // One launch over the matrices d[0 .. count) and, with hd, the head's TH
@@ -682,9 +707,12 @@ w4_status launch_rgroup(const w4r_desc* d, const RepackGeom* geo, int count, cud
   for (int i = 0; i < count; ++i) T += geo[i].ngroups;
   if (hd == nullptr) TH = 0;
   const int G = grid_of(T, TH, di);
+  RParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  split_by_rounds(geo, count, G, prm.cfirst);
   // every CTA stages the x of each matrix its range touches: split the
   // launch until that fits its shared memory
-  if (hd == nullptr && count > 1 && max_x_need(d, geo, count, T, G) > XCAP) {
+  if (hd == nullptr && count > 1 && max_x_need(d, geo, count, prm.cfirst, G) > XCAP) {
     const int h = count / 2;
     const w4_status rc = launch_rgroup(d, geo, h, st, di);
     if (rc != W4_OK) return rc;
@@ -692,8 +720,6 @@ w4_status launch_rgroup(const w4r_desc* d, const RepackGeom* geo, int count, cud
   }
   if ((T + TH) * G >= (int64_t(1) << 31))
     return fail(W4_ERR_SHAPE, "too many groups for one launch (%lld)", (long long)(T + TH));
-  RParams prm;
-  std::memset(&prm, 0, sizeof(prm));
   int g0 = 0;
   for (int i = 0; i < count; ++i) {
     RMat& m = prm.m[i];
@@ -875,7 +901,10 @@ w4_status decode_step(const w4r_desc* descs, int32_t count, const float* h, cons
   if (one_launch && n > 0) {
     int64_t T = 0;
     for (int i = 0; i < n; ++i) T += geo[i].ngroups;
-    one_launch = max_x_need(run, geo, n, T, grid_of(T, hg.ngroups, *di)) <= XCAP_STEP;
+    const int G = grid_of(T, hg.ngroups, *di);
+    static thread_local int32_t cfirst[GMAX + 1];
+    split_by_rounds(geo, n, G, cfirst);
+    one_launch = max_x_need(run, geo, n, cfirst, G) <= XCAP_STEP;
   }
   if (!one_launch) {
     // more matrices, x or h than one launch holds: the body's launches, then the head's

@@ -15,6 +15,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 @pytest.mark.parametrize("summary,algorithmic", [
     ("w4r_gemv_gpt2_m1.md", bench.body_bytes()),
     ("w4r_step_gpt2_m1.md", bench.body_bytes() + bench.head_bytes()),
+    ("w4r_gemv_3p8b_4layers_m1.md", 290193408),
+    ("w4_gemv_pageformat_3p8b_4layers_m8.md", 290193408),
     ("i8r_head_gpt2_m1.md", bench.head_bytes()),
     ("w4_gemv_pageformat_gpt2_m1.md", bench.body_bytes()),
     ("i8_rows_pageformat_gpt2_head_m1.md", bench.head_bytes()),
