@@ -478,20 +478,22 @@ def run_ours(args, world, rank, local):
 
 def run_e2e(wl, args, world, R):
     """Same step through the public binding with host buffers: per step, copy
-    the step's inputs from pinned host memory, run the step (one launch), read
-    every output back to pinned host memory."""
+    the step's inputs (the 48 x and h) from pinned host memory, run the step
+    (one launch), read the step's result, the logits, back to pinned host
+    memory. The body's outputs stay on the device, as a decoder's hidden
+    states do."""
     import torch
     stream = torch.cuda.current_stream()
     sh = int(stream.cuda_stream)
     inh = torch.from_numpy(wl.in_host).pin_memory()  # the 48 x and h, contiguous
-    outh = torch.empty(wl.out_dev.shape, dtype=torch.float32).pin_memory()  # the 48 y and the logits
+    outh = torch.empty(wl.logits.shape, dtype=torch.float32).pin_memory()  # the logits
     h2d = inh.numel() * 4
     d2h = outh.numel() * 4
 
     def step(r):
         wl.in_dev.copy_(inh, non_blocking=True)
         wl.step_fused(r, sh)
-        outh.copy_(wl.out_dev, non_blocking=True)
+        outh.copy_(wl.logits, non_blocking=True)
 
     for i in range(3):
         step(i % R)
