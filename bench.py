@@ -37,7 +37,7 @@ from int8_weight_quantized_w4_b200 import synth  # noqa: E402
 
 METRIC = "weight GB/s and decode tokens/s (GPT-2-small W4 stack, M=1) as % of HBM roofline"
 WORKLOAD = "gpt2-small W4 decode step: 48 body weights (12 x [768x2304, 768x768, 768x3072, 3072x768]) " \
-           "in one grouped launch + int8 tied head [768x50257] on the last position, M=1, fp32"
+           "+ int8 tied head [768x50257] on the last position, M=1, fp32"
 HEAD_K, HEAD_V = synth.GPT2_HIDDEN, synth.GPT2_VOCAB
 
 
