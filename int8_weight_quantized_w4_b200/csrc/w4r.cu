@@ -205,8 +205,9 @@ __device__ __forceinline__ void atom_m1(const uint8_t* st, int lane, const float
 }
 
 // The rounds one warp streams, in order: units u = warp + PW t of its CTA,
-// each a group of A rounds; unit u < nbc is body group lo + u, a later one
-// head group hlo + u - nbc. Producer (lane 0) and consumers walk the same
+// each a group of A rounds; in the fused step the CTA's nhc head groups come
+// first (unit u < nhc is head group hlo + u), then its body groups (unit u is
+// body group lo + u - nhc). Producer (lane 0) and consumers walk the same
 // sequence.
 struct RoundWalk {
   int t, r, ngw;  // unit ordinal of this warp, round in it, units of this warp
@@ -216,16 +217,16 @@ struct RoundWalk {
 };
 
 template <bool HEAD>
-__device__ __forceinline__ void walk_group(RoundWalk& w, const RParams& p, int lo, int nbc, int hlo, int warp) {
+__device__ __forceinline__ void walk_group(RoundWalk& w, const RParams& p, int lo, int nhc, int hlo, int warp) {
   const int u = warp + PW * w.t;
-  if (HEAD && u >= nbc) {
+  if (HEAD && u < nhc) {
     w.A = p.hd.A;
-    w.base = p.hd.tr + static_cast<int64_t>(hlo + u - nbc) * p.hd.group_bytes;
+    w.base = p.hd.tr + static_cast<int64_t>(hlo + u) * p.hd.group_bytes;
     w.rb = HROUND;
     w.last = HROUND + (32 << p.hd.gsl);  // the group's scales ride on its last round
     return;
   }
-  const int gg = lo + u;
+  const int gg = lo + u - nhc;
   while (w.g + 1 < p.count && p.m[w.g + 1].g0 <= gg) ++w.g;
   const RMat& m = p.m[w.g];
   w.A = ((m.K >> 5) << m.gsl) >> 5;
@@ -283,11 +284,11 @@ __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_co
     ++issued;
     if (++iw.r == iw.A) {
       iw.r = 0;
-      if (++iw.t < ngw) walk_group<HEAD>(iw, p, lo, nbc, hlo, warp);
+      if (++iw.t < ngw) walk_group<HEAD>(iw, p, lo, nhc, hlo, warp);
     }
   };
   if (ngw > 0) {
-    walk_group<HEAD>(iw, p, lo, nbc, hlo, warp);
+    walk_group<HEAD>(iw, p, lo, nhc, hlo, warp);
     if (lane == 0) {
       for (int s = 0; s < PST; ++s) mbar_init(&bar[s], 1);
       *abort_flag = 0;
@@ -345,9 +346,9 @@ __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_co
 #pragma unroll 1
   for (int t = 0; t < ngw && ok; ++t) {
     const int u = warp + PW * t;
-    if (HEAD && u >= nbc) {
+    if (HEAD && u < nhc) {
       // ---------------------------------------------------- a head group
-      const int hg = hlo + u - nbc;
+      const int hg = hlo + u;
       const int gsl = p.hd.gsl;
       const int gs = 1 << gsl;
       const int A = p.hd.A;
@@ -420,7 +421,7 @@ __global__ void __launch_bounds__(PW * 32, 1) w4r_gemv_m1_kernel(const __grid_co
       continue;
     }
     // ------------------------------------------------------ a body group
-    const int gg = lo + u;
+    const int gg = lo + u - nhc;
     while (g < glast && p.m[g + 1].g0 <= gg) {
       xo += p.m[g].K;
       ++g;
