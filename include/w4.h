@@ -422,8 +422,8 @@ W4_API w4_status i8r_head_argmax(const float* h, const void* tr, int64_t K, int6
  * w4r_matmul_grouped: repacked weights, M = 1) and the int8 head's logits
  * (as i8r_head_logits: logits[v] = s_v * sum_k h_k T[k, v] on the head in its
  * streaming layout), streamed by the same persistent CTAs, each of which takes
- * an equal share of the body's column groups and of the head's, so that the
- * step pays one launch's start and tail ("ONNX export, quantization and the
+ * an equal share of the head's column groups and of the body's bytes (the
+ * head's first), so that the step pays one launch's start and tail ("ONNX export, quantization and the
  * browser runtime", section "Quantization (train/quantize.py)", steps 2 to
  * 4). Every output is bit-identical to the two separate calls.
  * - descs / count: as for w4r_matmul_grouped (a HOST array, read during the
